@@ -1,0 +1,206 @@
+"""CPU oracle for the MoE router-and-dispatch path -- TEST INFRASTRUCTURE ONLY.
+
+The arithmetic lives in ``oracle.c`` (plain C, fp64, single-threaded); this
+module only compiles it with gcc and marshals numpy arrays.  Only ``tests/``,
+``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline / reference arm may
+import it.  It shares nothing with the CUDA library and the library never
+calls it.
+"""
+from __future__ import annotations
+
+import contextlib
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+SOFTMAX, SIGMOID, SQRT_SOFTPLUS, TOPK_SOFTMAX = 0, 1, 2, 3
+OK, ERR_ARG, ERR_INDEX, ERR_NAN = 0, 1, 4, 6
+
+_lib = None
+
+
+def compile_c(src: str, out: str) -> str:
+    """gcc an oracle source file into a shared library (ISO C, no FMA contraction)."""
+    tmp = out + f".tmp{os.getpid()}"
+    subprocess.check_call(
+        ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
+         "-o", tmp, src, "-lm"])
+    os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so next to its source if it is missing or stale."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        compile_c(_SRC, _LIB)
+    return _LIB
+
+
+@contextlib.contextmanager
+def using_library(path: str):
+    """Route every wrapper below through another build of the oracle (tests
+    use this to check that a planted mistake makes the pins fail)."""
+    global _lib
+    old = _lib
+    _lib = _bind(ctypes.CDLL(path))
+    try:
+        yield
+    finally:
+        _lib = old
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _bind(ctypes.CDLL(build()))
+    return _lib
+
+
+def _bind(lib):
+    P = ctypes.c_void_p
+    i32, i64, f64 = ctypes.c_int32, ctypes.c_int64, ctypes.c_double
+    lib.oracle_gate_rows.argtypes = [P, P, i32, i32, P, i64, P]
+    lib.oracle_gate_rows.restype = None
+    lib.oracle_scores.argtypes = [P, i64, i32, i32, P]
+    lib.oracle_scores.restype = None
+    lib.oracle_route.argtypes = [P, P, P, i64, i32, i32, i32, i32, i32, i32, i32, f64,
+                                 P, P, P, P]
+    lib.oracle_route.restype = ctypes.c_int
+    lib.oracle_weights_for_ids.argtypes = [P, P, i64, i32, i32, i32, i32, f64, P]
+    lib.oracle_weights_for_ids.restype = ctypes.c_int
+    lib.oracle_hash_route.argtypes = [P, P, i32, i32, P, i64, i32, i32, i32, f64, P, P]
+    lib.oracle_hash_route.restype = ctypes.c_int
+    lib.oracle_dispatch.argtypes = [P, i64, i32, i32, P, P, P, P]
+    lib.oracle_dispatch.restype = ctypes.c_int
+    lib.oracle_permute.argtypes = [P, P, i64, i32, i32, P]
+    lib.oracle_permute.restype = None
+    lib.oracle_combine.argtypes = [P, P, P, P, i64, i32, i32, P, P]
+    lib.oracle_combine.restype = None
+    return lib
+
+
+def _c(a, dtype):
+    """Contiguous array of the given dtype (no copy when already so)."""
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data
+
+
+def bf16_bits(a) -> np.ndarray:
+    """uint16 view of bf16 data given as a uint16 array or a torch bf16 tensor."""
+    if hasattr(a, "view") and hasattr(a, "dtype") and "bfloat16" in str(a.dtype):
+        import torch
+        return a.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    return _c(a, np.uint16)
+
+
+def gate_rows(x_bits, w_bits, rows=None) -> np.ndarray:
+    """fp64 logits of the listed rows: sum_i x[t,i]*W[e,i] in ascending i."""
+    x = _c(x_bits, np.uint16)
+    w = _c(w_bits, np.uint16)
+    T, d = x.shape
+    E = w.shape[0]
+    assert w.shape[1] == d
+    rows = np.arange(T, dtype=np.int64) if rows is None else _c(rows, np.int64)
+    out = np.empty((rows.size, E), np.float64)
+    _load().oracle_gate_rows(_p(x), _p(w), d, E, _p(rows), rows.size, _p(out))
+    return out
+
+
+def scores(logits, score: int) -> np.ndarray:
+    lg = _c(logits, np.float32)
+    T, E = lg.shape
+    out = np.empty((T, E), np.float64)
+    _load().oracle_scores(_p(lg), T, E, score, _p(out))
+    return out
+
+
+def route(logits, *, k_max, score, bias=None, k_per_token=None, n_groups=1, topk_groups=1,
+          group_topn=1, renormalize=True, route_scale=1.0, want_keys=False):
+    """Returns dict(ids, w, status[, keys, group_gap])."""
+    lg = _c(logits, np.float32)
+    T, E = lg.shape
+    b = None if bias is None else _c(bias, np.float32)
+    kp = None if k_per_token is None else _c(k_per_token, np.int32)
+    ids = np.empty((T, k_max), np.int32)
+    w = np.empty((T, k_max), np.float64)
+    keys = np.empty((T, E), np.float64) if want_keys else None
+    gap = np.empty((T,), np.float64) if want_keys else None
+    st = _load().oracle_route(_p(lg), _p(b), _p(kp), T, E, k_max, score, n_groups, topk_groups,
+                              group_topn, int(bool(renormalize)), float(route_scale), _p(ids),
+                              _p(w), _p(keys), _p(gap))
+    out = {"ids": ids, "w": w, "status": st}
+    if want_keys:
+        out["keys"] = keys
+        out["group_gap"] = gap
+    return out
+
+
+def weights_for_ids(logits, ids, *, score, renormalize=True, route_scale=1.0) -> np.ndarray:
+    lg = _c(logits, np.float32)
+    ids = _c(ids, np.int32)
+    T, E = lg.shape
+    k_max = ids.shape[1]
+    w = np.empty((T, k_max), np.float64)
+    st = _load().oracle_weights_for_ids(_p(lg), _p(ids), T, E, k_max, score,
+                                        int(bool(renormalize)), float(route_scale), _p(w))
+    assert st == OK, st
+    return w
+
+
+def hash_route(tok, table, *, num_experts, logits=None, score=SOFTMAX, renormalize=True,
+               route_scale=1.0):
+    tok = _c(tok, np.int32)
+    table = _c(table, np.int32)
+    vocab, k = table.shape
+    T = tok.shape[0]
+    lg = None if logits is None else _c(logits, np.float32)
+    ids = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    st = _load().oracle_hash_route(_p(tok), _p(table), vocab, k, _p(lg), T, num_experts, score,
+                                   int(bool(renormalize)), float(route_scale), _p(ids), _p(w))
+    return {"ids": ids, "w": w, "status": st}
+
+
+def dispatch(ids, num_experts):
+    ids = _c(ids, np.int32)
+    T, k_max = ids.shape
+    counts = np.empty((num_experts,), np.int32)
+    offsets = np.empty((num_experts + 1,), np.int32)
+    sorted_token = np.full((max(T * k_max, 1),), -7, np.int32)
+    dest_pos = np.empty((T, k_max), np.int32)
+    st = _load().oracle_dispatch(_p(ids), T, k_max, num_experts, _p(counts), _p(offsets),
+                                 _p(sorted_token), _p(dest_pos))
+    n = int(offsets[-1])
+    return {"counts": counts, "offsets": offsets, "sorted_token": sorted_token[:n],
+            "dest_pos": dest_pos, "status": st}
+
+
+def permute(x_bits, dest_pos, n_rows: int) -> np.ndarray:
+    x = _c(x_bits, np.uint16)
+    dp = _c(dest_pos, np.int32)
+    T, d = x.shape
+    xs = np.zeros((n_rows, d), np.uint16)
+    _load().oracle_permute(_p(x), _p(dp), T, dp.shape[1], d, _p(xs))
+    return xs
+
+
+def combine(y_bits, w, dest_pos, shared_bits=None, want_mag=True):
+    y = _c(y_bits, np.uint16)
+    wf = _c(w, np.float32)
+    dp = _c(dest_pos, np.int32)
+    T, k_max = dp.shape
+    d = y.shape[1]
+    sh = None if shared_bits is None else _c(shared_bits, np.uint16)
+    out = np.empty((T, d), np.float64)
+    mag = np.empty((T, d), np.float64) if want_mag else None
+    _load().oracle_combine(_p(y), _p(wf), _p(dp), _p(sh), T, k_max, d, _p(out), _p(mag))
+    return (out, mag) if want_mag else out
