@@ -1,0 +1,471 @@
+"""Benchmark of the B200 MoE router-and-dispatch path.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole path over one batch of synthetic tokens:
+gate GEMM -> route -> dispatch -> permute -> combine (the chain the workload
+defines), inputs resident in HBM.  L2 is flushed (a write larger than L2)
+before every timed step, outside the step's events.  Timing: CUDA events on the
+launching stream, barrier + synchronize around the K timed steps, max over
+ranks.  value = routed tokens/s of the whole job (T tokens per rank per step).
+
+Multi-GPU: the path shards by tokens with no exchange step, so each rank runs
+its own T-token batch (weak scaling, different seeds per rank, no collective in
+the data path; the only collectives are the barrier and the max-over-ranks of
+the timings).
+
+Extra keys: roofline (dominant kernel, algorithmic bytes / event time against
+the measured HBM copy bandwidth), stages (every kernel), clocks (nvidia-smi
+sampled during the timed steps), e2e (same metric through the C ABI with the
+inputs copied from pinned host memory and the output copied back inside the
+timed region), cpu_baseline (the fp64 CPU oracle on a bounded sample of the
+same workload), gpu_launches.
+
+--impl reference times the CPU oracle alone (the reference arm for this build:
+there is no upstream implementation to run), rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+DEFAULT_WORKLOAD = "qwen3_dynk"
+METRIC = "routed tokens/s (gate->top-k->permute->combine); % of HBM/tensor roofline"
+
+
+# ----------------------------------------------------------------- distributed
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    import datetime
+    if world > 1 and not torch.distributed.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.distributed.init_process_group(backend=backend,
+                                             timeout=datetime.timedelta(seconds=120))
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        if device is not None and torch.distributed.get_backend() == "nccl":
+            torch.distributed.barrier(device_ids=[device.index])
+        else:
+            torch.distributed.barrier()
+
+
+def reduce_max(value: float, world: int, device) -> float:
+    """Max of a per-rank float over all ranks (the job's time is its slowest rank)."""
+    if world == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, world: int, seconds_per_step_max: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's step time."""
+    return tokens_per_rank * world / seconds_per_step_max
+
+
+def rank_seed_offset(rank: int) -> int:
+    return 100000 * rank
+
+
+# ------------------------------------------------------------------ byte model
+def stage_bytes(wl, n_assign: int) -> dict:
+    """Algorithmic DRAM bytes per launch of each kernel (each read once, each
+    write once) and the gate's FLOPs."""
+    T, d, E, k = wl.T, wl.d, wl.E, wl.k_max
+    b = {}
+    if wl.gate:
+        b["gate_gemm"] = T * d * 2 + E * d * 2 + T * E * 4
+    b["route"] = T * E * 4 + T * k * 8 + (T * 4 if wl.k_choices else 0) + (E * 4 if wl.bias else 0)
+    b["dispatch"] = T * k * 4 + n_assign * 4 + T * k * 4 + 8 * E
+    b["permute"] = T * d * 2 + n_assign * d * 2 + T * k * 4
+    if wl.combine:
+        b["combine"] = n_assign * d * 2 + T * d * 2 + (T * d * 2 if wl.shared else 0) + 8 * T * k
+    return b
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get(
+            "bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "token_dispatch_moe_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the
+    current kernel sources; else None."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec.get("workloads", {}).get(workload, {}).get(kernel)
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- oracle chain
+def oracle_inputs(wl, inp: dict, n_tokens: int) -> dict:
+    """Host copies of the first n_tokens tokens of a workload's inputs, with
+    expert outputs for the sample's own assignments."""
+    from token_dispatch_moe_b200.workloads import normal_bf16
+
+    def bits(t):
+        return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+    h = {"T": n_tokens}
+    h["x"] = bits(inp["x"][:n_tokens])
+    h["w"] = bits(inp["w"]) if wl.gate else None
+    h["logits"] = inp["logits"][:n_tokens].cpu().numpy() if not wl.gate else None
+    h["bias"] = inp["bias"].cpu().numpy() if inp["bias"] is not None else None
+    kpt = inp["k_per_token"]
+    h["kpt"] = kpt[:n_tokens].cpu().numpy() if kpt is not None else None
+    n = int(h["kpt"].sum()) if kpt is not None else n_tokens * wl.k_max
+    h["y"] = bits(normal_bf16((max(n, 1), wl.d), 1.0, "cpu", 1000 * wl.index + 44))
+    h["shared"] = bits(inp["shared"][:n_tokens]) if inp["shared"] is not None else None
+    return h
+
+
+def oracle_chain(wl, h: dict) -> None:
+    """The path computed by the fp64 CPU oracle (single thread): gate, route,
+    dispatch, permute, combine, on the sample held in h."""
+    import oracle
+    score = {"softmax": oracle.SOFTMAX, "sigmoid": oracle.SIGMOID,
+             "sqrt_softplus": oracle.SQRT_SOFTPLUS, "topk_softmax": oracle.TOPK_SOFTMAX}[wl.score]
+    logits = oracle.gate_rows(h["x"], h["w"]).astype(np.float32) if wl.gate else h["logits"]
+    r = oracle.route(logits, k_max=wl.k_max, score=score, bias=h["bias"], k_per_token=h["kpt"],
+                     n_groups=wl.n_groups, topk_groups=wl.topk_groups, group_topn=wl.group_topn,
+                     renormalize=wl.renormalize, route_scale=wl.route_scale)
+    dsp = oracle.dispatch(r["ids"], wl.E)
+    n = int(dsp["offsets"][-1])
+    oracle.permute(h["x"], dsp["dest_pos"], n)
+    if wl.combine:
+        oracle.combine(h["y"][:max(n, 1)], r["w"].astype(np.float32), dsp["dest_pos"],
+                       h["shared"], want_mag=False)
+
+
+def oracle_sample_size(wl, inp, budget_s: float) -> int:
+    """Tokens of CPU work that take about budget_s seconds (calibrated on a small run)."""
+    n0 = min(64, wl.T)
+    h = oracle_inputs(wl, inp, n0)
+    t0 = time.perf_counter()
+    oracle_chain(wl, h)
+    per_token = (time.perf_counter() - t0) / n0
+    return int(max(8, min(wl.T, budget_s / max(per_token, 1e-9))))
+
+
+# ----------------------------------------------------------------- our arm
+def chain_launches(wl) -> int:
+    """Kernels of this library launched by one step of the chain."""
+    return (1 if wl.gate else 0) + 1 + 3 + 1 + (1 if wl.combine else 0)
+
+
+def run_ours(args):
+    world, rank, local = dist_env()
+    init_dist(world, "nccl")
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    import token_dispatch_moe_b200 as moe
+    from token_dispatch_moe_b200.path import RouterDispatch
+    from token_dispatch_moe_b200.workloads import WORKLOADS, make_inputs, num_assignments
+
+    moe.load_library()  # no fallback: fails loudly if the library is missing
+    wl = WORKLOADS[args.workload]
+    inp = make_inputs(wl, device, seed_offset=rank_seed_offset(rank))
+    n_assign = num_assignments(wl, inp["k_per_token"])
+    path = RouterDispatch(wl, device)
+    stream = torch.cuda.current_stream(device)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=device)
+    bytes_per = stage_bytes(wl, n_assign)
+    names = list(bytes_per)
+
+    def run_step(evs):
+        i = 0
+
+        def mark():
+            nonlocal i
+            if evs is not None:
+                evs[i].record(stream)
+                i += 1
+
+        mark()
+        logits = inp["logits"]
+        if wl.gate:
+            logits = path.gate(inp["x"], inp["w"])
+            mark()
+        path.route(logits, inp["bias"], inp["k_per_token"])
+        mark()
+        path.dispatch()
+        mark()
+        path.permute(inp["x"])
+        mark()
+        if wl.combine:
+            path.combine(inp["y"], inp["shared"])
+            mark()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        run_step(None)
+    torch.cuda.synchronize()
+    if path.status.item() != 0:
+        raise RuntimeError(f"device status {moe.moe_status_string(path.status.item())}")
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(K)]
+    with ClockSampler(device.index) as clk:
+        t_warm = time.perf_counter()
+        while time.perf_counter() - t_warm < 0.3:  # let the sampler start under load (untimed)
+            flush.zero_()
+            run_step(None)
+            torch.cuda.synchronize()
+        barrier(world, device)
+        torch.cuda.synchronize()
+        for s in range(K):
+            flush.zero_()  # L2 flush between timed steps, outside the step's events
+            run_step(evs[s])
+        torch.cuda.synchronize()
+        barrier(world, device)
+    step_ms = [evs[s][0].elapsed_time(evs[s][-1]) for s in range(K)]
+    stage_ms = {n: statistics.fmean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(K))
+                for i, n in enumerate(names)}
+    ms = statistics.fmean(step_ms)
+    ms_max = reduce_max(ms, world, device)
+    value = job_throughput(wl.T, world, ms_max / 1e3)
+
+    hbm, tf_burst, tf_sust, peak_kind = load_peaks()
+    stages = {}
+    for n in names:
+        gbs = bytes_per[n] / (stage_ms[n] / 1e3) / 1e9
+        stages[n] = {"us": round(stage_ms[n] * 1e3, 2), "bytes": bytes_per[n],
+                     "GB_s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4)}
+    if wl.gate:
+        flops = 2.0 * wl.T * wl.E * wl.d
+        stages["gate_gemm"]["TFLOP_s"] = round(flops / (stage_ms["gate_gemm"] / 1e3) / 1e12, 1)
+        stages["gate_gemm"]["frac_tensor"] = round(stages["gate_gemm"]["TFLOP_s"] / tf_sust, 4)
+    dom = max(stage_ms, key=stage_ms.get)
+    achieved = bytes_per[dom] / (stage_ms[dom] / 1e3) / 1e9
+    roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
+                "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                "traffic": recorded_traffic(wl.name, dom),
+                "algorithmic_bytes": bytes_per[dom], "peak_source": peak_kind}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(wl, inp, path, device, stream, min(K, args.e2e_steps), world)
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_max, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "tokens_per_gpu": wl.T, "hidden": wl.d, "experts": wl.E,
+                   "k": (f"{'/'.join(map(str, wl.k_choices))} per {wl.segment}-token request"
+                         if wl.k_choices else wl.k_max),
+                   "score": wl.score, "assignments_per_gpu": n_assign,
+                   "inputs": "bf16 x / W / expert outputs, fp32 logits",
+                   "l2": f"flushed before every timed step ({flush.numel() * 4 >> 20} MiB write)",
+                   "parallelism": f"token-sharded replicas x{world}"},
+        "roofline": roofline, "stages": stages, "clocks": clk.summary(),
+        "gpu_launches": chain_launches(wl) * K, "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(wl, inp, args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def measure_e2e(wl, inp, path, device, stream, steps, world):
+    """Same metric through the C ABI with host buffers: each step copies its
+    inputs from pinned host memory, runs the chain and copies the result back."""
+    names = [k for k in ("x", "w", "logits", "bias", "k_per_token", "y", "shared") if
+             inp[k] is not None]
+    host = {k: inp[k].cpu().pin_memory() for k in names}
+    dev = {k: torch.empty_like(inp[k]) for k in names}
+    full = dict(inp)
+    full.update(dev)
+    result_dev = path.out if wl.combine else path.xs
+    out_host = torch.empty(result_dev.shape, dtype=result_dev.dtype, pin_memory=True)
+    h2d = sum(host[k].numel() * host[k].element_size() for k in names)
+    d2h = out_host.numel() * out_host.element_size()
+
+    def one():
+        for k in names:
+            dev[k].copy_(host[k], non_blocking=True)
+        path.run(full)
+        out_host.copy_(result_dev, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world, device)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world, device)
+    ms = reduce_max(e0.elapsed_time(e1) / steps, world, device)
+    return {"value": round(job_throughput(wl.T, world, ms / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3),
+            "steps": steps}
+
+
+def cpu_baseline(wl, inp, budget_s: float) -> dict:
+    n = oracle_sample_size(wl, inp, budget_s)
+    h = oracle_inputs(wl, inp, n)
+    t0 = time.perf_counter()
+    oracle_chain(wl, h)
+    dt = time.perf_counter() - t0
+    return {"value": round(n / dt, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {n} of {wl.T} tokens of {wl.name}, full chain in fp64, "
+                      f"{dt:.1f} s on one host core"}
+
+
+# ---------------------------------------------------------- reference arm
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return  # the CPU oracle runs once, on rank 0
+    from token_dispatch_moe_b200.workloads import WORKLOADS, make_inputs
+    wl = WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_inputs(wl, dev, with_y=False)
+    total_budget = args.cpu_budget
+    per_step = oracle_sample_size(wl, inp, total_budget / max(1, args.steps + args.warmup))
+    h = oracle_inputs(wl, inp, per_step)
+    for _ in range(args.warmup):
+        oracle_chain(wl, h)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_chain(wl, h)
+    dt = time.perf_counter() - t0
+    value = per_step * args.steps / dt
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "tokens_per_step": per_step,
+                       "parallelism": "single host core"},
+            "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": 1,
+                             "kind": "oracle",
+                             "sample": f"first {per_step} of {wl.T} tokens per step"},
+            "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0,
+                    help="seconds of single-core oracle work for the CPU baseline")
+    args = ap.parse_args(argv)
+    world, _, _ = dist_env()
+    if world != args.gpus and not (world == 1 and args.gpus == 1):
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

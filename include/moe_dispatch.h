@@ -1,0 +1,204 @@
+/*
+ * moe_dispatch.h -- C ABI of the B200 (sm_100a) MoE router-and-dispatch library
+ * (libmoe_dispatch.so).
+ *
+ * The path, in call order on one CUDA stream:
+ *   moe_gate_gemm  -> fp32 gate logits = x . W^T on tcgen05 tensor cores
+ *   moe_route      -> score, selection-only bias, group limit, top-k with a
+ *                     per-token k, weights (renormalise, route_scale)
+ *   moe_hash_route -> (side path) expert ids looked up by token id
+ *   moe_dispatch   -> per-expert counts, offsets, stable expert-major order
+ *   moe_permute    -> hidden rows copied into expert-contiguous order
+ *   moe_combine    -> weighted fp32 sum of expert outputs back in token order,
+ *                     plus an optional shared expert
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers into memory the caller owns; the
+ *     library never allocates, frees or synchronises, and launches only on the
+ *     given stream.  Calls are asynchronous: outputs are ready when the stream
+ *     reaches them.
+ *   - Row-major layouts, no padding between rows.  bf16 tensors are passed as
+ *     moe_bf16_t (the raw 16-bit pattern).
+ *   - Host-side validation is synchronous: a bad argument returns a status and
+ *     launches nothing.  T = 0 is a valid no-op returning MOE_OK.
+ *   - d_status (where present, nullable) is a device int32 the caller zeroes;
+ *     kernels record the first device-side problem there (out-of-range id or
+ *     token, NaN logit, a wait that timed out) and never trap.  Read it after
+ *     the stream has synchronised.
+ *   - A failed launch returns MOE_ERR_CUDA after clearing the CUDA error.
+ *   - The library keeps no state between calls and is re-entrant.
+ *
+ * Sources, by page title and section:
+ *   "DeepSeek-V3.2-Exp - Select experts" (Explanation; gate-forward code
+ *     excerpt): fp32 gate linear, softmax/sigmoid, selection-only bias, group
+ *     limit, top-k, weights from unbiased scores, renormalise, route_scale.
+ *   "Crate ferrox_moe" (Functions; Structs RoutingDecision, MoeLayerConfig;
+ *     Enums GatingFunction): sqrt-softplus and gpt-oss scoring, norm_topk_prob,
+ *     route_hash, combine_expert_outputs.
+ *   "Feature Request: dynamic number of experts (hyperparam per request)": k
+ *     chosen per request from the same ranking.
+ *   "I modelli MoE open hanno router opposti": shared experts, hash-routed
+ *     first layers, expert counts and k of the model families.
+ */
+#ifndef MOE_DISPATCH_H
+#define MOE_DISPATCH_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so this header needs no CUDA
+ * headers.  NULL means the legacy default stream. */
+typedef struct CUstream_st *moe_stream_t;
+
+/* bf16 storage: the upper 16 bits of an IEEE binary32. */
+typedef uint16_t moe_bf16_t;
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,  /* host validation failed; nothing launched */
+    MOE_ERR_UNSUPPORTED = 2,  /* valid but outside this build's limits */
+    MOE_ERR_CUDA = 3,         /* a CUDA call or launch failed */
+    MOE_ERR_DEVICE_INDEX = 4, /* (d_status) id/token/k out of range seen on device */
+    MOE_ERR_TIMEOUT = 5,      /* (d_status) a bounded device wait gave up */
+    MOE_ERR_NAN_LOGIT = 6     /* (d_status) NaN logit seen; row still routed */
+} moe_status;
+
+/* Scoring functions.  "Crate ferrox_moe", Enums: GatingFunction. */
+typedef enum {
+    MOE_SCORE_SOFTMAX = 0,       /* softmax over all E, then top-k */
+    MOE_SCORE_SIGMOID = 1,       /* 1/(1+exp(-l)) per expert */
+    MOE_SCORE_SQRT_SOFTPLUS = 2, /* sqrt(log(1+exp(l))) per expert */
+    MOE_SCORE_TOPK_SOFTMAX = 3   /* gpt-oss: top-k on logits, softmax over those k */
+} moe_score_fn;
+
+/* Static per-layer routing configuration ("Crate ferrox_moe", MoeLayerConfig;
+ * the gate's constructor fields in "DeepSeek-V3.2-Exp - Select experts"). */
+typedef struct {
+    int32_t num_experts;  /* E: 1..512 */
+    int32_t k_max;        /* slots per token: 0..min(E, 32); per-token k <= k_max */
+    int32_t score;        /* moe_score_fn */
+    int32_t n_groups;     /* contiguous expert groups; 1 = no group limit; <= 32 */
+    int32_t topk_groups;  /* groups kept when n_groups > 1 */
+    int32_t group_topn;   /* group score = sum of its group_topn best keys: 1 (amax) or 2 */
+    int32_t renormalize;  /* nonzero: divide the selected weights by their sum */
+    float route_scale;    /* multiplies every weight (after renormalisation) */
+} moe_route_params;
+
+/* Human-readable name of a status code (static string). */
+const char *moe_status_string(moe_status s);
+
+/*
+ * moe_gate_gemm -- gate logits ("DeepSeek-V3.2-Exp - Select experts", gate
+ * forward: the linear layer computed in fp32).
+ *   logits[t][e] = sum_i x[t][i] * w[e][i]
+ * x      [T][d] bf16, w [E][d] bf16 (both K-major), logits [T][E] fp32 out.
+ * Products are exact in fp32 and accumulate in fp32 on tcgen05 tensor cores.
+ * Limits: 1 <= E <= 512, d >= 8 and d % 8 == 0 (16-byte rows), x, w 16-byte
+ * aligned, T * E < 2^31.  d_status (nullable) receives MOE_ERR_TIMEOUT if a
+ * pipeline wait exceeds its bound (it never should).
+ */
+moe_status moe_gate_gemm(const moe_bf16_t *x, const moe_bf16_t *w, float *logits, int64_t T,
+                         int32_t d, int32_t E, int32_t *d_status, moe_stream_t stream);
+
+/*
+ * moe_route -- scoring, selection and weights, one fused pass per token row.
+ * ("DeepSeek-V3.2-Exp - Select experts": Explanation and gate forward;
+ *  "Crate ferrox_moe": route_top_k_*; "Feature Request: dynamic number of
+ *  experts": per-request k.)
+ *   score s_e from the logit; selection key = s_e + bias[e] (bias nullable);
+ *   if n_groups > 1: group score = sum of the group_topn largest keys of each
+ *   contiguous group of E/n_groups experts, keep the topk_groups best groups;
+ *   take the k_t largest keys of kept experts (k_t = k_per_token[t], or k_max
+ *   if k_per_token is NULL), in descending key order, equal keys -> lower id;
+ *   weight = unbiased s_e (gpt-oss: softmax over the k_t selected logits),
+ *   divided by their sum if renormalize, times route_scale.
+ * logits [T][E] fp32; bias [E] fp32 or NULL; k_per_token [T] int32 or NULL.
+ * Out: topk_ids [T][k_max] int32 (-1 in slots >= k_t), topk_w [T][k_max] fp32
+ * (0 in those slots).
+ * Validation: E % n_groups == 0, k_max <= topk_groups * E / n_groups,
+ * group_topn in {1, 2} and <= E / n_groups.  On the device a k_per_token value
+ * outside [0, k_max] is clamped and reported as MOE_ERR_DEVICE_INDEX; a NaN
+ * logit ranks below every number and is reported as MOE_ERR_NAN_LOGIT.
+ */
+moe_status moe_route(const float *logits, const float *bias, const int32_t *k_per_token,
+                     const moe_route_params *params, int64_t T, int32_t *topk_ids,
+                     float *topk_w, int32_t *d_status, moe_stream_t stream);
+
+/*
+ * moe_hash_route -- expert ids from a token-id table ("Crate ferrox_moe",
+ * route_hash: the DeepSeek-V4 hash layers look the ids up by token id; no
+ * bias, no selection).
+ *   topk_ids[t][j] = tid2eid[token_ids[t]][j]  (a repeated id keeps both slots)
+ * tid2eid [vocab][k] int32, row-major (ggml's [k, vocab]); k <= 32.
+ * Weights: with logits [T][E] given, the score (params->score) of each looked-up
+ * expert, then renormalize / route_scale as in moe_route; with logits NULL,
+ * route_scale / k per slot.  params->num_experts = E; other fields of params
+ * besides score, renormalize and route_scale are ignored.
+ * A token id outside [0, vocab) empties its row (ids -1, weights 0); a table
+ * entry outside [0, E) empties its slot; both report MOE_ERR_DEVICE_INDEX.
+ */
+moe_status moe_hash_route(const int32_t *token_ids, const int32_t *tid2eid, int32_t vocab,
+                          int32_t k, const float *logits, const moe_route_params *params,
+                          int64_t T, int32_t *topk_ids, float *topk_w, int32_t *d_status,
+                          moe_stream_t stream);
+
+/*
+ * moe_dispatch_workspace_size -- bytes of device scratch moe_dispatch needs for
+ * T tokens, k_max slots and E experts (depends only on T*k_max and E).
+ */
+moe_status moe_dispatch_workspace_size(int64_t T, int32_t k_max, int32_t E, size_t *bytes);
+
+/*
+ * moe_dispatch -- histogram, exclusive scan and stable scatter of the
+ * assignments into expert-contiguous order (the dispatch step that makes
+ * "only the selected experts process the input" concrete).
+ *   counts[e]   = number of slots with id e;
+ *   offsets[0]  = 0, offsets[e+1] = offsets[e] + counts[e]  (offsets[E] = N);
+ *   walking slots in flat order a = t*k_max + j (slots with id -1 skipped),
+ *   pos = offsets[e] + number of earlier slots with the same e;
+ *   sorted_token[pos] = t, dest_pos[a] = pos (-1 for empty slots).
+ * topk_ids [T][k_max]; counts [E]; offsets [E+1]; sorted_token capacity
+ * T*k_max (the first N entries are written); dest_pos [T][k_max].
+ * workspace: ws_bytes >= moe_dispatch_workspace_size(), 256-byte aligned; its
+ * contents need no initialisation.  T*k_max < 2^31.  An id outside [-1, E) is
+ * treated as empty and reported as MOE_ERR_DEVICE_INDEX.
+ */
+moe_status moe_dispatch(const int32_t *topk_ids, int64_t T, int32_t k_max, int32_t E,
+                        int32_t *counts, int32_t *offsets, int32_t *sorted_token,
+                        int32_t *dest_pos, void *workspace, size_t ws_bytes, int32_t *d_status,
+                        moe_stream_t stream);
+
+/*
+ * moe_permute -- xs[dest_pos[t][j]] = x[t] for every slot with dest_pos >= 0
+ * (a bit-exact row copy into expert-contiguous order).  Token-major: each row
+ * of x is read once and written to its k_t destinations.
+ * x [T][d] bf16; dest_pos [T][k_max] from moe_dispatch; xs [N][d] bf16.
+ * d % 8 == 0; x and xs 16-byte aligned.
+ */
+moe_status moe_permute(const moe_bf16_t *x, const int32_t *dest_pos, int64_t T, int32_t k_max,
+                       int32_t d, moe_bf16_t *xs, moe_stream_t stream);
+
+/*
+ * moe_combine -- weighted sum of expert outputs back in token order
+ * ("Crate ferrox_moe", combine_expert_outputs: routed plus shared).
+ *   out[t] = bf16_rne( sum_{j: dest_pos[t][j] >= 0} topk_w[t][j] * y[dest_pos[t][j]]
+ *                      + shared[t] )
+ * accumulated in fp32 in slot order j = 0, 1, ..., the shared expert (unit
+ * weight, nullable) added last.
+ * y [N][d] bf16 (expert outputs in expert-contiguous order); topk_w,
+ * dest_pos [T][k_max]; shared [T][d] bf16 or NULL; out [T][d] bf16.
+ * d % 8 == 0; y, shared, out 16-byte aligned.
+ */
+moe_status moe_combine(const moe_bf16_t *y, const float *topk_w, const int32_t *dest_pos,
+                       const moe_bf16_t *shared, int64_t T, int32_t k_max, int32_t d,
+                       moe_bf16_t *out, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_DISPATCH_H */

@@ -1,0 +1,92 @@
+"""The C-ABI library without a GPU: it builds for sm_100a, loads, exports
+every entry point include/*.h declares, and its host-side validation answers
+with status codes before any CUDA call."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import token_dispatch_moe_b200 as moe
+from token_dispatch_moe_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = build_mod.build()
+    return moe.load_library(path)
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(moe_\w+)\s*\(", text, flags=re.M))
+    return sorted(names)
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for n in ("moe_gate_gemm", "moe_route", "moe_hash_route", "moe_dispatch",
+              "moe_dispatch_workspace_size", "moe_permute", "moe_combine", "moe_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_status_strings(lib):
+    assert moe.moe_status_string(0) == "ok"
+    assert "timed out" in moe.moe_status_string(moe.MOE_ERR_TIMEOUT)
+
+
+def test_workspace_size(lib):
+    # one int32 per (segment, expert); segments of 32 * items slots, rounded to 256 B
+    assert moe.moe_dispatch_workspace_size(0, 8, 256) == 0
+    b = moe.moe_dispatch_workspace_size(16384, 16, 128)
+    n_flat = 16384 * 16
+    assert b >= (n_flat // (32 * 64)) * 128 * 4 and b % 256 == 0
+    assert moe.moe_dispatch_workspace_size(1, 1, 1) == 256
+    with pytest.raises(moe.MoeError):
+        moe.moe_dispatch_workspace_size(10, 33, 8)   # k_max > 32
+    with pytest.raises(moe.MoeError):
+        moe.moe_dispatch_workspace_size(10, 4, 513)  # E > 512
+
+
+def test_host_validation_needs_no_gpu(lib):
+    P = moe.RouteParams
+    bad = ctypes.c_void_p(16)  # never dereferenced: validation fails first
+    # route: NULL params, E % n_groups, k > kept experts, bad score, k_max > 32
+    assert lib.moe_route(bad, None, None, None, 4, bad, bad, None, None) == moe.MOE_ERR_INVALID_ARG
+    for p in (P.make(12, 4, "softmax", n_groups=5), P.make(12, 4, "softmax", n_groups=4),
+              P.make(12, 4, 7), P.make(64, 33, "softmax"), P.make(600, 4, "softmax"),
+              P.make(16, 2, "sigmoid", n_groups=4, topk_groups=2, group_topn=3)):
+        assert lib.moe_route(bad, None, None, ctypes.byref(p), 4, bad, bad, None, None) != 0
+    # T = 0 is a no-op that returns OK without touching the device
+    p = P.make(12, 4, "softmax")
+    assert lib.moe_route(None, None, None, ctypes.byref(p), 0, None, None, None, None) == 0
+    assert lib.moe_gate_gemm(bad, bad, bad, 4, 12, 8, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_gate_gemm(bad, bad, bad, 4, 64, 513, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_gate_gemm(None, None, None, 0, 64, 8, None, None) == 0
+    assert lib.moe_hash_route(bad, bad, 10, 0, None, ctypes.byref(p), 4, bad, bad, None,
+                              None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_permute(bad, bad, 4, 2, 12, bad, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(bad, bad, bad, None, 4, 2, 10, bad, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_permute(ctypes.c_void_p(18), bad, 4, 2, 16, bad, None) == \
+        moe.MOE_ERR_INVALID_ARG  # x not 16-byte aligned
+    ws = ctypes.c_void_p(256 * 3 + 8)  # not 256-byte aligned
+    assert lib.moe_dispatch(bad, 4, 2, 8, bad, bad, bad, bad, ws, 1 << 20, None, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_dispatch(bad, 4, 2, 8, bad, bad, bad, bad, ctypes.c_void_p(256), 0, None,
+                            None) == moe.MOE_ERR_INVALID_ARG  # workspace too small
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    with pytest.raises(RuntimeError, match="missing"):
+        moe.load_library(str(tmp_path / "libmoe_dispatch.so"))

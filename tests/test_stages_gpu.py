@@ -1,0 +1,279 @@
+"""Stage-by-stage parity of the CUDA path with the oracle on small and edge
+shapes: ragged tiles, scalar and vector layouts, maximum sizes, empty inputs,
+ties, NaN, out-of-range ids.  All calls go through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import token_dispatch_moe_b200 as moe
+from gpu_check import (bits, check_combine, check_dispatch, check_gate, check_permute,
+                       check_route)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _gen(seed):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(seed)
+    return g
+
+
+def _status():
+    return torch.zeros(1, dtype=torch.int32, device=DEV)
+
+
+# ------------------------------------------------------------------ gate GEMM
+@pytest.mark.parametrize("T,d,E", [(1, 64, 128), (300, 200, 8), (257, 2048, 128),
+                                   (129, 512, 30), (200, 1024, 256), (131, 7168, 384),
+                                   (140, 256, 512), (128, 8, 16), (333, 128, 300)])
+def test_gate_gemm_integer_exact(T, d, E):
+    """Integer-valued x, W in [-4, 4]: every product and partial sum is exact in
+    fp32, so the logits must equal the oracle bit for bit whatever the order."""
+    g = _gen(T * 7 + d + E)
+    x = torch.randint(-4, 5, (T, d), generator=g, device=DEV).to(torch.bfloat16)
+    w = torch.randint(-4, 5, (E, d), generator=g, device=DEV).to(torch.bfloat16)
+    logits = torch.full((T, E), float("nan"), device=DEV)
+    st = _status()
+    moe.moe_gate_gemm(x, w, logits, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    o = oracle.gate_rows(bits(x), bits(w))
+    assert np.array_equal(logits.cpu().numpy().astype(np.float64), o)
+
+
+@pytest.mark.parametrize("T,d,E", [(515, 2048, 128), (300, 7168, 256), (260, 7168, 384)])
+def test_gate_gemm_random(T, d, E):
+    g = _gen(T + d + E)
+    x = torch.randn((T, d), generator=g, device=DEV).to(torch.bfloat16)
+    w = (torch.randn((E, d), generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    logits = torch.empty((T, E), device=DEV)
+    moe.moe_gate_gemm(x, w, logits)
+    torch.cuda.synchronize()
+    check_gate(logits, x, w)
+
+
+def test_gate_gemm_validation():
+    x = torch.zeros((4, 12), dtype=torch.bfloat16, device=DEV)
+    w = torch.zeros((4, 12), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(moe.MoeError):
+        moe.moe_gate_gemm(x, w, torch.empty((4, 4), device=DEV))  # d % 8 != 0
+    x = torch.zeros((0, 64), dtype=torch.bfloat16, device=DEV)
+    moe.moe_gate_gemm(x, torch.zeros((4, 64), dtype=torch.bfloat16, device=DEV),
+                      torch.empty((0, 4), device=DEV))  # T = 0 is a no-op
+
+
+# ---------------------------------------------------------------------- route
+ROUTE_CASES = [
+    # E, k_max, score, bias, G, TG, topn, renorm, scale, dyn
+    (8, 2, "softmax", False, 1, 1, 1, True, 1.0, False),
+    (128, 16, "softmax", False, 1, 1, 1, True, 1.0, True),
+    (128, 8, "softmax", False, 1, 1, 1, False, 1.0, False),
+    (256, 8, "sigmoid", True, 8, 4, 2, True, 2.5, False),
+    (256, 8, "sigmoid", False, 8, 4, 1, True, 1.0, False),
+    (384, 6, "sqrt_softplus", False, 1, 1, 1, True, 1.0, False),
+    (384, 6, "sqrt_softplus", True, 4, 2, 2, True, 1.5, False),
+    (128, 1, "sigmoid", False, 1, 1, 1, False, 1.0, False),
+    (128, 4, "topk_softmax", False, 1, 1, 1, True, 1.0, False),
+    (128, 4, "topk_softmax", True, 1, 1, 1, False, 1.0, False),
+    (30, 5, "softmax", True, 3, 2, 2, True, 1.0, True),      # scalar layout, odd groups
+    (7, 7, "sigmoid", False, 1, 1, 1, True, 1.0, False),      # k = E
+    (512, 32, "softmax", False, 1, 1, 1, True, 1.0, False),   # maximum E and k
+    (512, 32, "sigmoid", True, 32, 8, 2, True, 1.0, True),    # 32 groups of 16
+    (96, 12, "sqrt_softplus", False, 6, 4, 2, False, 2.0, True),
+]
+
+
+@pytest.mark.parametrize("case", ROUTE_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_route_parity(case):
+    E, k_max, score, has_bias, G, TG, topn, renorm, scale, dyn = case
+    T = 1003
+    g = _gen(E * 31 + k_max)
+    logits = torch.randn((T, E), generator=g, device=DEV) * 2
+    logits[::17] = torch.round(logits[::17] * 2) / 2  # rows with many exact ties
+    logits[5] = 0.0                                   # a row where every key ties
+    bias = (torch.rand((E,), generator=g, device=DEV) * 0.2 - 0.1) if has_bias else None
+    kpt = torch.randint(0, k_max + 1, (T,), generator=g, device=DEV,
+                        dtype=torch.int32) if dyn else None
+    p = moe.RouteParams.make(E, k_max, score, G, TG, topn, renorm, scale)
+    ids = torch.full((T, k_max), -7, dtype=torch.int32, device=DEV)
+    w = torch.full((T, k_max), 7.0, device=DEV)
+    st = _status()
+    moe.moe_route(logits, bias, kpt, p, ids, w, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    r = check_route(ids.cpu().numpy(), w.cpu().numpy(), logits.cpu().numpy(), k_max=k_max,
+                    score=score, bias=None if bias is None else bias.cpu().numpy(),
+                    kpt=None if kpt is None else kpt.cpu().numpy(), n_groups=G, topk_groups=TG,
+                    group_topn=topn, renormalize=renorm, route_scale=scale)
+    print(case, r)
+
+
+def test_route_nan_and_bad_k():
+    E, k = 16, 4
+    logits = torch.randn((3, E), device=DEV)
+    logits[1, 3] = float("nan")
+    kpt = torch.tensor([2, 4, 9], dtype=torch.int32, device=DEV)  # 9 > k_max: clamped
+    p = moe.RouteParams.make(E, k, "sigmoid", renormalize=False)
+    ids = torch.empty((3, k), dtype=torch.int32, device=DEV)
+    w = torch.empty((3, k), device=DEV)
+    st = _status()
+    moe.moe_route(logits, None, kpt, p, ids, w, st)
+    torch.cuda.synchronize()
+    assert st.item() in (moe.MOE_ERR_NAN_LOGIT, moe.MOE_ERR_DEVICE_INDEX)
+    assert 3 not in ids[1].tolist()  # NaN ranks below every number
+    assert (ids[2] >= 0).all()       # clamped to k_max
+    assert (ids[0, 2:] == -1).all() and (w[0, 2:] == 0).all()
+
+
+def test_route_validation():
+    logits = torch.zeros((2, 12), device=DEV)
+    ids = torch.empty((2, 4), dtype=torch.int32, device=DEV)
+    w = torch.empty((2, 4), device=DEV)
+    for p in (moe.RouteParams.make(12, 4, "softmax", n_groups=5, topk_groups=1),  # E % G
+              moe.RouteParams.make(12, 4, "softmax", n_groups=4, topk_groups=1),  # k > kept
+              moe.RouteParams.make(12, 4, 9)):                                    # bad score
+        with pytest.raises(moe.MoeError):
+            moe.moe_route(logits, None, None, p, ids, w)
+    moe.moe_route(torch.zeros((0, 12), device=DEV), None, None,
+                  moe.RouteParams.make(12, 4, "softmax"), ids[:0], w[:0])
+
+
+# ----------------------------------------------------------------- hash route
+@pytest.mark.parametrize("score,with_logits,renorm", [("sqrt_softplus", True, True),
+                                                      ("softmax", True, False),
+                                                      ("softmax", True, True),
+                                                      ("topk_softmax", True, True),
+                                                      ("sigmoid", False, True)])
+def test_hash_route_parity(score, with_logits, renorm):
+    T, E, k, vocab = 777, 384, 6, 5000
+    g = _gen(99)
+    tok = torch.randint(0, vocab, (T,), generator=g, device=DEV, dtype=torch.int32)
+    table = torch.randint(0, E, (vocab, k), generator=g, device=DEV, dtype=torch.int32)
+    table[tok[0]] = torch.tensor([3, 3, 5, 3, 9, 1], dtype=torch.int32, device=DEV)
+    logits = torch.randn((T, E), generator=g, device=DEV) if with_logits else None
+    p = moe.RouteParams.make(E, k, score, renormalize=renorm, route_scale=1.25)
+    ids = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, k), device=DEV)
+    st = _status()
+    moe.moe_hash_route(tok, table, logits, p, ids, w, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    o = oracle.hash_route(tok.cpu().numpy(), table.cpu().numpy(), num_experts=E,
+                          logits=None if logits is None else logits.cpu().numpy(),
+                          score=oracle_score(score), renormalize=renorm, route_scale=1.25)
+    assert np.array_equal(ids.cpu().numpy(), o["ids"])
+    wg = w.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(wg - o["w"]) <= 1e-5 * np.abs(o["w"]))
+
+
+def oracle_score(name):
+    return {"softmax": oracle.SOFTMAX, "sigmoid": oracle.SIGMOID,
+            "sqrt_softplus": oracle.SQRT_SOFTPLUS, "topk_softmax": oracle.TOPK_SOFTMAX}[name]
+
+
+def test_hash_route_bad_entries():
+    E, k, vocab = 16, 3, 10
+    tok = torch.tensor([1, 10, 2, -1], dtype=torch.int32, device=DEV)
+    table = torch.randint(0, E, (vocab, k), device=DEV, dtype=torch.int32)
+    table[2, 1] = E  # out of range slot
+    p = moe.RouteParams.make(E, k, "softmax")
+    ids = torch.empty((4, k), dtype=torch.int32, device=DEV)
+    w = torch.empty((4, k), device=DEV)
+    st = _status()
+    moe.moe_hash_route(tok, table, None, p, ids, w, st)
+    torch.cuda.synchronize()
+    assert st.item() == moe.MOE_ERR_DEVICE_INDEX
+    o = oracle.hash_route(tok.cpu().numpy(), table.cpu().numpy(), num_experts=E)
+    assert np.array_equal(ids.cpu().numpy(), o["ids"])
+    assert np.allclose(w.cpu().numpy(), o["w"], rtol=1e-6, atol=0)
+
+
+# ------------------------------------------------------------------- dispatch
+def _dispatch(ids, E):
+    T, k = ids.shape
+    counts = torch.full((E,), -5, dtype=torch.int32, device=DEV)
+    offsets = torch.full((E + 1,), -5, dtype=torch.int32, device=DEV)
+    st_tok = torch.full((max(T * k, 1),), -5, dtype=torch.int32, device=DEV)
+    dest = torch.full((T, k), -5, dtype=torch.int32, device=DEV)
+    ws = torch.full((max(moe.moe_dispatch_workspace_size(T, k, E), 256),), 0xAB,
+                    dtype=torch.uint8, device=DEV)  # garbage: no initialisation needed
+    st = _status()
+    moe.moe_dispatch(ids, E, counts, offsets, st_tok, dest, ws, st)
+    torch.cuda.synchronize()
+    return counts, offsets, st_tok, dest, st.item()
+
+
+@pytest.mark.parametrize("T,k,E,empty_frac,hot", [
+    (1, 1, 1, 0.0, False), (1000, 8, 256, 0.0, False), (3001, 4, 128, 0.0, True),
+    (777, 16, 128, 0.4, False), (5000, 6, 384, 0.0, False), (20000, 32, 512, 0.1, True),
+    (333, 3, 7, 0.2, False), (70000, 8, 256, 0.0, True)])
+def test_dispatch_parity(T, k, E, empty_frac, hot):
+    g = _gen(T + k + E)
+    ids = torch.randint(0, E, (T, k), generator=g, device=DEV, dtype=torch.int32)
+    if hot:  # skewed load: a third of the slots on two experts
+        m = torch.rand((T, k), generator=g, device=DEV) < 0.33
+        ids[m] = torch.randint(0, 2, (int(m.sum()),), generator=g, device=DEV,
+                               dtype=torch.int32) * (E - 1)
+    if empty_frac:
+        ids[torch.rand((T, k), generator=g, device=DEV) < empty_frac] = -1
+    counts, offsets, st_tok, dest, st = _dispatch(ids, E)
+    assert st == 0
+    check_dispatch(ids.cpu().numpy(), counts.cpu().numpy(), offsets.cpu().numpy(),
+                   st_tok.cpu().numpy(), dest.cpu().numpy(), E)
+
+
+def test_dispatch_edge_cases():
+    for ids in (torch.full((5, 3), -1, dtype=torch.int32, device=DEV),  # all empty
+                torch.zeros((6, 0), dtype=torch.int32, device=DEV),     # k_max = 0
+                torch.zeros((0, 4), dtype=torch.int32, device=DEV)):    # T = 0
+        counts, offsets, st_tok, dest, st = _dispatch(ids, 9)
+        assert st == 0
+        assert (counts == 0).all() and (offsets == 0).all()
+        if ids.numel():
+            assert (dest == -1).all()
+    ids = torch.tensor([[0, 9], [3, -2], [1, 1]], dtype=torch.int32, device=DEV)
+    counts, offsets, st_tok, dest, st = _dispatch(ids, 4)
+    assert st == moe.MOE_ERR_DEVICE_INDEX
+    o = oracle.dispatch(ids.cpu().numpy(), 4)
+    assert np.array_equal(dest.cpu().numpy(), o["dest_pos"])
+    assert np.array_equal(counts.cpu().numpy(), o["counts"])
+
+
+# ---------------------------------------------------------- permute / combine
+@pytest.mark.parametrize("T,k,d,E", [(1, 1, 8, 4), (999, 8, 2048, 64), (500, 6, 7168, 384),
+                                     (1234, 4, 2880, 128), (100, 32, 136, 512),
+                                     (257, 2, 128, 8)])
+def test_permute_combine_parity(T, k, d, E):
+    g = _gen(T * 3 + d)
+    ids = torch.randint(0, E, (T, k), generator=g, device=DEV, dtype=torch.int32)
+    ids[::9, k - 1] = -1  # some empty slots
+    counts, offsets, st_tok, dest, st = _dispatch(ids, E)
+    n = int(offsets[-1].item())
+    x = torch.randn((T, d), generator=g, device=DEV).to(torch.bfloat16)
+    xs = torch.zeros((max(n, 1), d), dtype=torch.bfloat16, device=DEV)
+    moe.moe_permute(x, dest, xs)
+    torch.cuda.synchronize()
+    check_permute(xs, x, dest.cpu().numpy())
+    y = torch.randn((max(n, 1), d), generator=g, device=DEV).to(torch.bfloat16)
+    w = torch.rand((T, k), generator=g, device=DEV) * (dest >= 0)
+    for shared in (None, torch.randn((T, d), generator=g, device=DEV).to(torch.bfloat16)):
+        out = torch.empty((T, d), dtype=torch.bfloat16, device=DEV)
+        moe.moe_combine(y, w, dest, shared, out)
+        torch.cuda.synchronize()
+        check_combine(out, y, w.cpu().numpy(), dest.cpu().numpy(), shared)
+
+
+def test_permute_combine_validation():
+    x = torch.zeros((4, 17), dtype=torch.bfloat16, device=DEV)
+    dest = torch.zeros((4, 2), dtype=torch.int32, device=DEV)
+    xs = torch.zeros((8, 16), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(moe.MoeError):  # x not 16-byte aligned (offset by one element)
+        moe.moe_permute(x.view(-1)[1:65].view(4, 16), dest, xs)
+    out = torch.zeros((4, 16), dtype=torch.bfloat16, device=DEV)
+    sh = torch.ones((4, 16), dtype=torch.bfloat16, device=DEV)
+    moe.moe_combine(xs, torch.zeros((4, 0), device=DEV),
+                    torch.zeros((4, 0), dtype=torch.int32, device=DEV), sh, out)
+    torch.cuda.synchronize()
+    assert torch.equal(out, sh)  # k_max = 0: the shared expert alone

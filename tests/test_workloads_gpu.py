@@ -1,0 +1,85 @@
+"""Parity of the whole chain on every workload, through the same RouterDispatch
+object the benchmark times.
+
+* reduced: the workload's d, E, k and scoring with a ragged token count the
+  oracle finishes in seconds; every output of every stage is checked.
+* full: the workload at its full size; route and dispatch are checked on every
+  row, the gate, permute and combine on sampled tokens (first, last, random).
+Each stage's oracle is fed the GPU's previous-stage output.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gpu_check import (check_combine, check_dispatch, check_gate, check_permute, check_route,
+                       np32)
+from token_dispatch_moe_b200.path import RouterDispatch
+from token_dispatch_moe_b200.workloads import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+REDUCED_T = {"mixtral_tiny": 253, "qwen3_dynk": 1500, "deepseek_v3": 777,
+             "deepseek_v4": 777, "llama4_top1": 3001, "gptoss_top4": 3001}
+
+
+def _sample(T, n, seed):
+    rng = np.random.default_rng(seed)
+    pick = rng.choice(T, size=min(n, T), replace=False)
+    return np.unique(np.concatenate([pick, [0, T - 1]]))
+
+
+def _run_and_check(wl, sampled: bool):
+    inp = make_inputs(wl, "cuda")
+    path = RouterDispatch(wl)
+    path.run(inp)
+    torch.cuda.synchronize()
+    assert path.status.item() == 0, path.status.item()
+    report = {}
+    logits = path.logits if wl.gate else inp["logits"]
+    if wl.gate:
+        rows = _sample(wl.T, 192, 1) if sampled else None
+        report["gate_worst"] = check_gate(logits, inp["x"], inp["w"], rows)
+    ids, w = np32(path.topk_ids), np32(path.topk_w)
+    report["route"] = check_route(ids, w, np32(logits), k_max=wl.k_max, score=wl.score,
+                                  bias=np32(inp["bias"]), kpt=np32(inp["k_per_token"]),
+                                  n_groups=wl.n_groups, topk_groups=wl.topk_groups,
+                                  group_topn=wl.group_topn, renormalize=wl.renormalize,
+                                  route_scale=wl.route_scale)
+    dest = np32(path.dest_pos)
+    n = check_dispatch(ids, np32(path.counts), np32(path.offsets), np32(path.sorted_token), dest,
+                       wl.E)
+    tokens = _sample(wl.T, 1024, 2) if sampled else None
+    check_permute(path.xs, inp["x"], dest, tokens)
+    if wl.combine:
+        assert inp["y"].shape[0] == n
+        tokens = _sample(wl.T, 512, 3) if sampled else None
+        report["combine_worst"] = check_combine(path.out, inp["y"], w, dest, inp["shared"], tokens)
+    if wl.hash_vocab:
+        path.run_hash_layer(inp, logits)
+        torch.cuda.synchronize()
+        assert path.status.item() == 0
+        import oracle
+        o = oracle.hash_route(np32(inp["token_ids"]), np32(inp["tid2eid"]), num_experts=wl.E,
+                              logits=np32(logits), score=oracle.SQRT_SOFTPLUS,
+                              renormalize=wl.renormalize, route_scale=wl.route_scale)
+        hid = np32(path.hash_ids)
+        assert np.array_equal(hid, o["ids"])
+        hw = np32(path.hash_w).astype(np.float64)
+        assert np.all(np.abs(hw - o["w"]) <= 1e-5 * np.abs(o["w"]))
+        hdest = np32(path.dest_pos)
+        check_dispatch(hid, np32(path.counts), np32(path.offsets), np32(path.sorted_token),
+                       hdest, wl.E)
+        check_permute(path.xs, inp["x"], hdest, _sample(wl.T, 1024, 4) if sampled else None)
+    print(wl.name, wl.T, report)
+    return report
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_workload_reduced(name):
+    _run_and_check(WORKLOADS[name].scaled(REDUCED_T[name]), sampled=False)
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_workload_full(name):
+    _run_and_check(WORKLOADS[name], sampled=True)
+    torch.cuda.empty_cache()

@@ -1,0 +1,69 @@
+// Internal helpers of libmoe_dispatch (device side and launch plumbing).
+// Every kernel of the library includes this; nothing outside the library does.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe_dispatch.h"
+
+#define MOE_FULL_MASK 0xffffffffu
+
+namespace moe {
+
+inline cudaStream_t as_cuda(moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Map the outcome of the launches just issued to a status, clearing the error.
+inline moe_status launch_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+inline int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+    return n > 0 ? n : 148;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// First device-side problem wins; later ones are dropped.
+__device__ __forceinline__ void report(int32_t *status, int32_t code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+// Order-preserving map of an fp32 value to uint32: a larger float gives a
+// larger key; -0 and +0 give the same key; NaN gives 1, below every number
+// (-inf maps to 0x007fffff); 0 is reserved for "not selectable".
+__device__ __forceinline__ uint32_t order_key(float v) {
+    if (v != v) return 1u;
+    uint32_t u = __float_as_uint(v == 0.0f ? 0.0f : v);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(MOE_FULL_MASK, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(MOE_FULL_MASK, v, o));
+    return v;
+}
+
+// Per-expert scores that do not depend on the rest of the row.
+__device__ __forceinline__ float sigmoid_score(float l) { return 1.0f / (1.0f + expf(-l)); }
+__device__ __forceinline__ float sqrt_softplus_score(float l) {
+    return sqrtf(fmaxf(l, 0.0f) + log1pf(expf(-fabsf(l))));
+}
+
+// Streaming loads for data read exactly once.
+__device__ __forceinline__ float4 ld_stream(const float4 *p) { return __ldcs(p); }
+__device__ __forceinline__ float ld_stream(const float *p) { return __ldcs(p); }
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p) { return __ldcs(p); }
+
+}  // namespace moe

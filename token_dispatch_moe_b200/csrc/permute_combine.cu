@@ -1,0 +1,176 @@
+// moe_permute and moe_combine: the two HBM-bound row movers of the path.
+//
+// permute: xs[dest_pos[t][j]] = x[t]   (bit-exact copy into expert order)
+// combine: out[t] = bf16_rne( sum_j w[t][j] * y[dest_pos[t][j]] + shared[t] ),
+//          fp32 accumulation in slot order, the shared expert ("Crate
+//          ferrox_moe", combine_expert_outputs: routed + shared) added last.
+//
+// B200 design: both kernels are token-major, one warp per token row, 16-byte
+// vector accesses.  permute reads each row of x once and writes it to its k_t
+// destinations (T*d*2 + N*d*2 bytes: the algorithmic minimum; a gather loop
+// over destination rows would re-read x k times).  combine gathers the k_t
+// expert rows of a token and writes one row; loads of four slots are issued
+// before their FMAs so that enough bytes are in flight per warp.
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kRowWarps = 8;
+
+__device__ __forceinline__ void fma_bf16x8(float *acc, float w, const uint4 &v) {
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        acc[2 * i] = fmaf(w, __uint_as_float(u[i] << 16), acc[2 * i]);
+        acc[2 * i + 1] = fmaf(w, __uint_as_float(u[i] & 0xffff0000u), acc[2 * i + 1]);
+    }
+}
+
+__device__ __forceinline__ void add_bf16x8(float *acc, const uint4 &v) {
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        acc[2 * i] += __uint_as_float(u[i] << 16);
+        acc[2 * i + 1] += __uint_as_float(u[i] & 0xffff0000u);
+    }
+}
+
+__device__ __forceinline__ uint4 pack_bf16x8(const float *acc) {
+    uint32_t u[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+        u[i] = *reinterpret_cast<uint32_t *>(&h);
+    }
+    return make_uint4(u[0], u[1], u[2], u[3]);
+}
+
+template <int U>
+__global__ void __launch_bounds__(kRowWarps * 32)
+    permute_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ dest_pos, int64_t T,
+                   int k_max, int nvec, uint4 *__restrict__ xs) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nw = (int64_t)gridDim.x * kRowWarps;
+    for (int64_t row = (int64_t)blockIdx.x * kRowWarps + (threadIdx.x >> 5); row < T; row += nw) {
+        const int dp = lane < k_max ? dest_pos[row * k_max + lane] : -1;
+        const uint4 *src = x + row * nvec;
+        for (int v0 = 0; v0 < nvec; v0 += 32 * U) {
+            uint4 buf[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int v = v0 + u * 32 + lane;
+                if (v < nvec) buf[u] = ld_stream(src + v);
+            }
+            for (int j = 0; j < k_max; ++j) {
+                const int pos = __shfl_sync(MOE_FULL_MASK, dp, j);
+                if (pos < 0) continue;
+                uint4 *dst = xs + (int64_t)pos * nvec;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    if (v < nvec) dst[v] = buf[u];
+                }
+            }
+        }
+    }
+}
+
+template <int U>
+__global__ void __launch_bounds__(kRowWarps * 32)
+    combine_kernel(const uint4 *__restrict__ y, const float *__restrict__ w,
+                   const int32_t *__restrict__ dest_pos, const uint4 *__restrict__ shared,
+                   int64_t T, int k_max, int nvec, uint4 *__restrict__ out) {
+    constexpr int J = 4;  // slots whose loads are issued together
+    const int lane = threadIdx.x & 31;
+    const int64_t nw = (int64_t)gridDim.x * kRowWarps;
+    for (int64_t row = (int64_t)blockIdx.x * kRowWarps + (threadIdx.x >> 5); row < T; row += nw) {
+        const int dp = lane < k_max ? dest_pos[row * k_max + lane] : -1;
+        const float wl = lane < k_max ? w[row * k_max + lane] : 0.0f;
+        for (int v0 = 0; v0 < nvec; v0 += 32 * U) {
+            float acc[U][8];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[u][i] = 0.0f;
+            for (int j0 = 0; j0 < k_max; j0 += J) {
+                int pos[J];
+                float wt[J];
+                uint4 t[J][U];
+#pragma unroll
+                for (int q = 0; q < J; ++q) {
+                    const int j = j0 + q;
+                    pos[q] = __shfl_sync(MOE_FULL_MASK, dp, j & 31);
+                    wt[q] = __shfl_sync(MOE_FULL_MASK, wl, j & 31);
+                    if (j >= k_max) pos[q] = -1;
+                }
+#pragma unroll
+                for (int q = 0; q < J; ++q)
+                    if (pos[q] >= 0) {
+                        const uint4 *src = y + (int64_t)pos[q] * nvec;
+#pragma unroll
+                        for (int u = 0; u < U; ++u) {
+                            const int v = v0 + u * 32 + lane;
+                            t[q][u] = v < nvec ? ld_stream(src + v) : make_uint4(0, 0, 0, 0);
+                        }
+                    }
+#pragma unroll
+                for (int q = 0; q < J; ++q)
+                    if (pos[q] >= 0)
+#pragma unroll
+                        for (int u = 0; u < U; ++u) fma_bf16x8(acc[u], wt[q], t[q][u]);
+            }
+            if (shared) {
+                const uint4 *src = shared + row * nvec;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    if (v < nvec) add_bf16x8(acc[u], ld_stream(src + v));
+                }
+            }
+            uint4 *dst = out + row * nvec;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int v = v0 + u * 32 + lane;
+                if (v < nvec) dst[v] = pack_bf16x8(acc[u]);
+            }
+        }
+    }
+}
+
+unsigned row_grid(int64_t T) {
+    const int64_t need = (T + kRowWarps - 1) / kRowWarps;
+    const int64_t cap = (int64_t)sm_count() * 32;
+    return (unsigned)(need < cap ? need : cap);
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" moe_status moe_permute(const moe_bf16_t *x, const int32_t *dest_pos, int64_t T,
+                                  int32_t k_max, int32_t d, moe_bf16_t *xs, moe_stream_t stream) {
+    using namespace moe;
+    if (T < 0 || k_max < 0 || k_max > 32 || d < 8 || d % 8 != 0) return MOE_ERR_INVALID_ARG;
+    if (T == 0 || k_max == 0) return MOE_OK;
+    if (!x || !dest_pos || !xs || !aligned16(x) || !aligned16(xs)) return MOE_ERR_INVALID_ARG;
+    if (T * (int64_t)k_max >= (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+    permute_kernel<8><<<row_grid(T), kRowWarps * 32, 0, as_cuda(stream)>>>(
+        reinterpret_cast<const uint4 *>(x), dest_pos, T, k_max, d / 8,
+        reinterpret_cast<uint4 *>(xs));
+    return launch_status();
+}
+
+extern "C" moe_status moe_combine(const moe_bf16_t *y, const float *topk_w,
+                                  const int32_t *dest_pos, const moe_bf16_t *shared, int64_t T,
+                                  int32_t k_max, int32_t d, moe_bf16_t *out, moe_stream_t stream) {
+    using namespace moe;
+    if (T < 0 || k_max < 0 || k_max > 32 || d < 8 || d % 8 != 0) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!out || !aligned16(out) || (shared && !aligned16(shared))) return MOE_ERR_INVALID_ARG;
+    if (k_max > 0 && (!y || !topk_w || !dest_pos || !aligned16(y))) return MOE_ERR_INVALID_ARG;
+    if (T * (int64_t)k_max >= (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+    combine_kernel<2><<<row_grid(T), kRowWarps * 32, 0, as_cuda(stream)>>>(
+        reinterpret_cast<const uint4 *>(y), topk_w, dest_pos,
+        reinterpret_cast<const uint4 *>(shared), T, k_max, d / 8, reinterpret_cast<uint4 *>(out));
+    return launch_status();
+}

@@ -1,0 +1,85 @@
+"""The router-and-dispatch chain as one object: buffers plus the C-ABI calls in
+order (gate -> route -> dispatch -> permute -> combine), all on one stream.
+
+Only orchestration lives here: torch allocates device memory, and every step
+is a call into libmoe_dispatch.so.  The expert FFN between permute and combine
+is outside the path; its outputs ``y`` are an input of :meth:`RouterDispatch.run`.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (RouteParams, moe_combine, moe_dispatch, moe_dispatch_workspace_size,
+               moe_gate_gemm, moe_hash_route, moe_permute, moe_route)
+from .workloads import Workload
+
+
+class RouterDispatch:
+    """Preallocated buffers for T tokens of one layer configuration."""
+
+    def __init__(self, wl: Workload, device="cuda", n_rows: int | None = None):
+        self.wl = wl
+        self.params = RouteParams.make(wl.E, wl.k_max, wl.score, wl.n_groups, wl.topk_groups,
+                                       wl.group_topn, wl.renormalize, wl.route_scale)
+        T, E, k = wl.T, wl.E, wl.k_max
+        i32 = dict(dtype=torch.int32, device=device)
+        self.logits = torch.empty((T, E), dtype=torch.float32, device=device) if wl.gate else None
+        self.topk_ids = torch.empty((T, k), **i32)
+        self.topk_w = torch.empty((T, k), dtype=torch.float32, device=device)
+        self.counts = torch.empty((E,), **i32)
+        self.offsets = torch.empty((E + 1,), **i32)
+        self.sorted_token = torch.empty((max(T * k, 1),), **i32)
+        self.dest_pos = torch.empty((T, k), **i32)
+        ws = moe_dispatch_workspace_size(T, k, E)
+        self.workspace = torch.empty((max(ws, 256),), dtype=torch.uint8, device=device)
+        rows = T * k if n_rows is None else n_rows
+        self.xs = torch.empty((max(rows, 1), wl.d), dtype=torch.bfloat16, device=device)
+        self.out = (torch.empty((T, wl.d), dtype=torch.bfloat16, device=device)
+                    if wl.combine else None)
+        self.status = torch.zeros((1,), **i32)
+        if wl.hash_vocab:
+            self.hash_ids = torch.empty((T, k), **i32)
+            self.hash_w = torch.empty((T, k), dtype=torch.float32, device=device)
+
+    # Individual steps (each one C-ABI call) -----------------------------------
+    def gate(self, x, w, stream=None):
+        moe_gate_gemm(x, w, self.logits, self.status, stream)
+        return self.logits
+
+    def route(self, logits, bias=None, k_per_token=None, stream=None):
+        moe_route(logits, bias, k_per_token, self.params, self.topk_ids, self.topk_w,
+                  self.status, stream)
+
+    def hash_route(self, token_ids, tid2eid, logits=None, stream=None):
+        moe_hash_route(token_ids, tid2eid, logits, self.params, self.hash_ids, self.hash_w,
+                       self.status, stream)
+
+    def dispatch(self, ids=None, stream=None):
+        moe_dispatch(self.topk_ids if ids is None else ids, self.wl.E, self.counts, self.offsets,
+                     self.sorted_token, self.dest_pos, self.workspace, self.status, stream)
+
+    def permute(self, x, stream=None):
+        moe_permute(x, self.dest_pos, self.xs, stream)
+
+    def combine(self, y, shared=None, stream=None):
+        moe_combine(y, self.topk_w, self.dest_pos, shared, self.out, stream)
+
+    # The whole chain -----------------------------------------------------------
+    def run(self, inputs: dict, stream=None):
+        """gate (if the workload has one) -> route -> dispatch -> permute ->
+        combine (if the workload ends there).  ``inputs`` as made by
+        :func:`workloads.make_inputs`."""
+        logits = self.gate(inputs["x"], inputs["w"], stream) if self.wl.gate else inputs["logits"]
+        self.route(logits, inputs["bias"], inputs["k_per_token"], stream)
+        self.dispatch(stream=stream)
+        self.permute(inputs["x"], stream)
+        if self.wl.combine:
+            self.combine(inputs["y"], inputs["shared"], stream)
+        return self.out if self.wl.combine else self.xs
+
+    def run_hash_layer(self, inputs: dict, logits=None, stream=None):
+        """hash_route -> dispatch -> permute (the hash-routed layer's chain)."""
+        self.hash_route(inputs["token_ids"], inputs["tid2eid"], logits, stream)
+        self.dispatch(self.hash_ids, stream)
+        self.permute(inputs["x"], stream)
+        return self.xs
