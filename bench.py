@@ -27,6 +27,7 @@ there is no upstream implementation to run), rank 0 only.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -266,29 +267,30 @@ def run_ours(args):
     bytes_per = stage_bytes(wl, n_assign)
     names = list(bytes_per)
 
-    def run_step(evs):
+    def run_step(mark):
+        """One pass of the chain; mark(i) records the i-th stage boundary."""
         i = 0
 
-        def mark():
+        def boundary():
             nonlocal i
-            if evs is not None:
-                evs[i].record(stream)
-                i += 1
+            if mark is not None:
+                mark(i)
+            i += 1
 
-        mark()
+        boundary()
         logits = inp["logits"]
         if wl.gate:
             logits = path.gate(inp["x"], inp["w"])
-            mark()
+            boundary()
         path.route(logits, inp["bias"], inp["k_per_token"])
-        mark()
+        boundary()
         path.dispatch()
-        mark()
+        boundary()
         path.permute(inp["x"])
-        mark()
+        boundary()
         if wl.combine:
             path.combine(inp["y"], inp["shared"])
-            mark()
+            boundary()
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -298,7 +300,47 @@ def run_ours(args):
         raise RuntimeError(f"device status {moe.moe_status_string(path.status.item())}")
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(K)]
+    nb = len(names) + 1
+    if args.eager:
+        # Stream launches, one set of events per step.
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nb)] for _ in range(K)]
+        cur = {"s": 0}
+
+        def mark(i):
+            evs[cur["s"]][i].record(stream)
+
+        def timed_step(s):
+            cur["s"] = s
+            run_step(mark)
+    else:
+        # The step captured once as a CUDA graph (no host launch overhead);
+        # stage boundaries are event-record nodes inside it, read after each replay.
+        gev = [torch.cuda.Event(enable_timing=True) for _ in range(nb)]
+        for e in gev:
+            e.record(stream)
+        torch.cuda.synchronize()
+        cudart = ctypes.CDLL("libcudart.so.12")
+        cudart.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p,
+                                                    ctypes.c_uint]
+        cap = torch.cuda.Stream(device)
+
+        def mark(i):
+            err = cudart.cudaEventRecordWithFlags(gev[i].cuda_event, cap.cuda_stream, 1)
+            if err != 0:
+                raise RuntimeError(f"cudaEventRecordWithFlags failed ({err})")
+
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap, capture_error_mode="relaxed"):
+            run_step(mark)
+        graph.replay()
+        torch.cuda.synchronize()
+        times = []
+
+        def timed_step(s):
+            graph.replay()
+            torch.cuda.synchronize()
+            times.append([gev[0].elapsed_time(gev[i]) for i in range(nb)])
+
     with ClockSampler(device.index) as clk:
         t_warm = time.perf_counter()
         while time.perf_counter() - t_warm < 0.3:  # let the sampler start under load (untimed)
@@ -309,12 +351,15 @@ def run_ours(args):
         torch.cuda.synchronize()
         for s in range(K):
             flush.zero_()  # L2 flush between timed steps, outside the step's events
-            run_step(evs[s])
+            timed_step(s)
         torch.cuda.synchronize()
         barrier(world, device)
-    step_ms = [evs[s][0].elapsed_time(evs[s][-1]) for s in range(K)]
-    stage_ms = {n: statistics.fmean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(K))
-                for i, n in enumerate(names)}
+    if args.eager:
+        marks = [[evs[s][0].elapsed_time(evs[s][i]) for i in range(nb)] for s in range(K)]
+    else:
+        marks = times
+    step_ms = [m[-1] for m in marks]
+    stage_ms = {n: statistics.fmean(m[i + 1] - m[i] for m in marks) for i, n in enumerate(names)}
     ms = statistics.fmean(step_ms)
     ms_max = reduce_max(ms, world, device)
     value = job_throughput(wl.T, world, ms_max / 1e3)
@@ -351,7 +396,8 @@ def run_ours(args):
                    "score": wl.score, "assignments_per_gpu": n_assign,
                    "inputs": "bf16 x / W / expert outputs, fp32 logits",
                    "l2": f"flushed before every timed step ({flush.numel() * 4 >> 20} MiB write)",
-                   "parallelism": f"token-sharded replicas x{world}"},
+                   "parallelism": f"token-sharded replicas x{world}",
+                   "launch": "stream (eager)" if args.eager else "CUDA graph of the step"},
         "roofline": roofline, "stages": stages, "clocks": clk.summary(),
         "gpu_launches": chain_launches(wl) * K, "e2e": e2e,
     }
@@ -452,6 +498,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch from the host every step instead of replaying a CUDA graph")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
