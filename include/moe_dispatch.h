@@ -173,6 +173,29 @@ moe_status moe_dispatch(const int32_t *topk_ids, int64_t T, int32_t k_max, int32
                         moe_stream_t stream);
 
 /*
+ * moe_dispatch_static -- moe_dispatch without a caller-provided workspace.
+ * (No counterpart in the source pages: this entry point exists for callers that
+ * cannot allocate device memory, e.g. a plugin running inside a host framework
+ * that owns every device allocation, or code that must avoid the implicit
+ * device synchronisation of cudaMalloc.)
+ * Same arguments, outputs and status rules as moe_dispatch, minus workspace and
+ * ws_bytes.  Its scratch is a 4 MiB array inside the library, held by every GPU
+ * that loads the library until the process exits; sizes whose
+ * moe_dispatch_workspace_size() exceeds 4 MiB are rejected with
+ * MOE_ERR_UNSUPPORTED and nothing is launched.  The library allocates and frees
+ * nothing here either.
+ * The first call on a device (made with that device current) looks up the
+ * scratch array's device address; make that first call before any stream
+ * capture.  All calls share the one array: two calls whose work overlaps on
+ * the GPU (different streams, or different host threads) race and give wrong
+ * results; serialise them.  The array keeps the last call's contents, but no
+ * call depends on them: everything a call reads from it, it wrote first.
+ */
+moe_status moe_dispatch_static(const int32_t *topk_ids, int64_t T, int32_t k_max, int32_t E,
+                               int32_t *counts, int32_t *offsets, int32_t *sorted_token,
+                               int32_t *dest_pos, int32_t *d_status, moe_stream_t stream);
+
+/*
  * moe_permute -- xs[dest_pos[t][j]] = x[t] for every slot with dest_pos >= 0
  * (a bit-exact row copy into expert-contiguous order).  Token-major: each row
  * of x is read once and written to its k_t destinations.

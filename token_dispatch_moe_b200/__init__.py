@@ -22,7 +22,8 @@ __all__ = [
     "MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED", "MOE_ERR_CUDA",
     "MOE_ERR_DEVICE_INDEX", "MOE_ERR_TIMEOUT", "MOE_ERR_NAN_LOGIT",
     "moe_status_string", "moe_gate_gemm", "moe_route", "moe_hash_route",
-    "moe_dispatch_workspace_size", "moe_dispatch", "moe_permute", "moe_combine",
+    "moe_dispatch_workspace_size", "moe_dispatch", "moe_dispatch_static", "moe_permute",
+    "moe_combine",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -83,6 +84,7 @@ def load_library(path: str | None = None):
         "moe_hash_route": ([P, P, i32, i32, P, ctypes.POINTER(RouteParams), i64, P, P, P, P], st),
         "moe_dispatch_workspace_size": ([i64, i32, i32, ctypes.POINTER(ctypes.c_size_t)], st),
         "moe_dispatch": ([P, i64, i32, i32, P, P, P, P, P, ctypes.c_size_t, P, P], st),
+        "moe_dispatch_static": ([P, i64, i32, i32, P, P, P, P, P, P], st),
         "moe_permute": ([P, P, i64, i32, i32, P, P], st),
         "moe_combine": ([P, P, P, P, i64, i32, i32, P, P], st),
     }
@@ -202,6 +204,26 @@ def moe_dispatch(topk_ids, E, counts, offsets, sorted_token, dest_pos, workspace
                                        _ptr(sorted_token), _ptr(dest_pos), _ptr(workspace),
                                        workspace.numel(), _ptr(d_status), _stream(stream)),
            "moe_dispatch")
+
+
+def moe_dispatch_static(topk_ids, E, counts, offsets, sorted_token, dest_pos, d_status=None,
+                        stream=None):
+    """moe_dispatch with the library's own fixed 4 MiB scratch instead of a
+    caller-allocated workspace, for callers that cannot allocate device memory.
+    Calls that overlap on the GPU race on that scratch; the first call on a
+    device should come before any stream capture."""
+    _need(topk_ids, torch.int32, "topk_ids", 2)
+    for t, n in ((counts, "counts"), (offsets, "offsets"), (sorted_token, "sorted_token"),
+                 (dest_pos, "dest_pos"), (d_status, "d_status")):
+        _need(t, torch.int32, n)
+    T, k_max = topk_ids.shape
+    if counts.numel() < E or offsets.numel() < E + 1 or sorted_token.numel() < T * k_max or \
+            tuple(dest_pos.shape) != (T, k_max):
+        raise ValueError("shape mismatch")
+    _check(load_library().moe_dispatch_static(_ptr(topk_ids), T, k_max, E, _ptr(counts),
+                                              _ptr(offsets), _ptr(sorted_token), _ptr(dest_pos),
+                                              _ptr(d_status), _stream(stream)),
+           "moe_dispatch_static")
 
 
 def moe_permute(x, dest_pos, xs, stream=None):

@@ -20,6 +20,8 @@
 //               (popcount of lower lanes in the match mask) and writes
 //               sorted_token and dest_pos.
 // The workspace is seg: S x E int32, S = ceil(T*k_max / SEG).
+#include <atomic>
+
 #include "common.cuh"
 
 namespace moe {
@@ -205,4 +207,52 @@ extern "C" moe_status moe_dispatch(const int32_t *topk_ids, int64_t T, int32_t k
         }
     }
     return launch_status();
+}
+
+// ------------------------------------------------- dispatch, no caller scratch
+// A variant of moe_dispatch for callers that cannot allocate device memory
+// themselves.  Its scratch is this file-scope device array: every GPU that
+// loads the library holds these 4 MiB until the process exits.  Host code must
+// not pass the array's name to a kernel (on the host it is only a stand-in);
+// the device address is fetched with cudaGetSymbolAddress once per device and
+// cached.
+namespace moe {
+namespace {
+constexpr size_t kStaticScratchBytes = size_t(4) << 20;
+constexpr int kMaxDevices = 64;
+std::atomic<void *> g_static_scratch_addr[kMaxDevices];
+}  // namespace
+}  // namespace moe
+
+static __device__ __align__(256) int32_t g_dispatch_scratch[moe::kStaticScratchBytes / sizeof(int32_t)];
+
+extern "C" moe_status moe_dispatch_static(const int32_t *topk_ids, int64_t T, int32_t k_max,
+                                          int32_t E, int32_t *counts, int32_t *offsets,
+                                          int32_t *sorted_token, int32_t *dest_pos,
+                                          int32_t *d_status, moe_stream_t stream) {
+    using namespace moe;
+    size_t need = 0;
+    moe_status st = moe_dispatch_workspace_size(T, k_max, E, &need);
+    if (st != MOE_OK) return st;
+    if (need > kStaticScratchBytes) return MOE_ERR_UNSUPPORTED;  // beyond the fixed scratch
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+    void *addr = g_static_scratch_addr[dev].load(std::memory_order_acquire);
+    if (!addr) {
+        // First call on this device (with it current): resolve the array's
+        // device address.  Two threads racing here store the same value.
+        if (cudaGetSymbolAddress(&addr, g_dispatch_scratch) != cudaSuccess || !addr) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
+        g_static_scratch_addr[dev].store(addr, std::memory_order_release);
+    }
+    // Every scratch entry a dispatch reads is written earlier by the same
+    // dispatch, so the array needs no clearing between calls.
+    return moe_dispatch(topk_ids, T, k_max, E, counts, offsets, sorted_token, dest_pos, addr,
+                        kStaticScratchBytes, d_status, stream);
 }
