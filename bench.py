@@ -258,6 +258,8 @@ def run_ours(args):
 
     moe.load_library()  # no fallback: fails loudly if the library is missing
     wl = WORKLOADS[args.workload]
+    if args.tokens:
+        wl = wl.scaled(args.tokens)
     inp = make_inputs(wl, device, seed_offset=rank_seed_offset(rank))
     n_assign = num_assignments(wl, inp["k_per_token"])
     path = RouterDispatch(wl, device)
@@ -390,7 +392,8 @@ def run_ours(args):
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_max, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
         "data": "synthetic",
-        "config": {"workload": wl.name, "tokens_per_gpu": wl.T, "hidden": wl.d, "experts": wl.E,
+        "config": {"workload": wl.name if not args.tokens else f"{wl.name}@T={wl.T}",
+                   "tokens_per_gpu": wl.T, "hidden": wl.d, "experts": wl.E,
                    "k": (f"{'/'.join(map(str, wl.k_choices))} per {wl.segment}-token request"
                          if wl.k_choices else wl.k_max),
                    "score": wl.score, "assignments_per_gpu": n_assign,
@@ -497,6 +500,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the workload's token count (profiling of smaller cases)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--eager", action="store_true",
                     help="launch from the host every step instead of replaying a CUDA graph")

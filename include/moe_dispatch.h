@@ -116,7 +116,8 @@ moe_status moe_gate_gemm(const moe_bf16_t *x, const moe_bf16_t *w, float *logits
  *   if k_per_token is NULL), in descending key order, equal keys -> lower id;
  *   weight = unbiased s_e (gpt-oss: softmax over the k_t selected logits),
  *   divided by their sum if renormalize, times route_scale.
- * logits [T][E] fp32; bias [E] fp32 or NULL; k_per_token [T] int32 or NULL.
+ * logits [T][E] fp32, 16-byte aligned; bias [E] fp32 or NULL; k_per_token [T]
+ * int32 or NULL.
  * Out: topk_ids [T][k_max] int32 (-1 in slots >= k_t), topk_w [T][k_max] fp32
  * (0 in those slots).
  * Validation: E % n_groups == 0, k_max <= topk_groups * E / n_groups,

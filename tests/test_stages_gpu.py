@@ -138,6 +138,9 @@ def test_route_validation():
             moe.moe_route(logits, None, None, p, ids, w)
     moe.moe_route(torch.zeros((0, 12), device=DEV), None, None,
                   moe.RouteParams.make(12, 4, "softmax"), ids[:0], w[:0])
+    with pytest.raises(moe.MoeError):  # logits not 16-byte aligned
+        moe.moe_route(torch.zeros((2 * 12 + 1,), device=DEV)[1:].view(2, 12), None, None,
+                      moe.RouteParams.make(12, 4, "softmax"), ids, w)
 
 
 # ----------------------------------------------------------------- hash route
@@ -277,3 +280,25 @@ def test_permute_combine_validation():
                     torch.zeros((4, 0), dtype=torch.int32, device=DEV), sh, out)
     torch.cuda.synchronize()
     assert torch.equal(out, sh)  # k_max = 0: the shared expert alone
+
+
+@pytest.mark.parametrize("k_max,score,has_bias", [(1, "sigmoid", False), (4, "topk_softmax", False),
+                                                  (8, "softmax", True), (16, "softmax", False)])
+def test_route_keys_equal_in_high_bits(k_max, score, has_bias):
+    """Rows whose keys differ only in their lowest mantissa bits: any scheme
+    that compares shortened keys must still reach the exact selection."""
+    T, E = 515, 128
+    g = _gen(777 + k_max)
+    base = torch.randn((T, 1), generator=g, device=DEV) * 2
+    steps = torch.randint(-40, 41, (T, E), generator=g, device=DEV).float()
+    logits = (base * (1 + steps * 2.0 ** -21)).contiguous()  # neighbours a few ulps apart
+    logits[::3, 5] = logits[::3, 9]                          # and some exact ties
+    bias = (torch.rand((E,), generator=g, device=DEV) * 1e-6) if has_bias else None
+    p = moe.RouteParams.make(E, k_max, score)
+    ids = torch.empty((T, k_max), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, k_max), device=DEV)
+    moe.moe_route(logits, bias, None, p, ids, w)
+    torch.cuda.synchronize()
+    r = check_route(ids.cpu().numpy(), w.cpu().numpy(), logits.cpu().numpy(), k_max=k_max,
+                    score=score, bias=None if bias is None else bias.cpu().numpy())
+    print(r)

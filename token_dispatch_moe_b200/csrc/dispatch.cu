@@ -6,20 +6,22 @@
 // pos = offsets[e] + (number of earlier slots with id e); sorted_token[pos] = t,
 // dest_pos[a] = pos (-1 for empty slots).
 //
-// B200 design: three short launches and no inter-block waiting.
-//   1. count:   each warp owns a segment of SEG consecutive slots and builds its
-//               segment's histogram in shared memory with warp-aggregated
-//               updates (__match_any_sync: one leader per distinct id adds the
-//               popcount of its peers) -> seg[s][e] in the workspace.
-//   2. scan:    per expert, exclusive prefix of seg[.][e] over segments (in
-//               place) and the total counts[e]; 32 experts per block so every
-//               row access is a coalesced 128-byte line.
-//   3. scatter: each block scans counts into offsets in shared memory (block 0
-//               also writes them out); each warp walks its segment again in
-//               order, ranks every slot among its peers with the same id
+// B200 design: two short launches, no inter-block waiting.  The slots are cut
+// into S block segments of 8 warps x W items x 32 lanes, each warp owning a
+// contiguous sub-segment.
+//   1. count:   every warp builds its sub-segment's histogram in shared memory
+//               with warp-aggregated updates (__match_any_sync: one leader per
+//               distinct id adds the popcount of its peers) and stores it; the
+//               block also stores its segment's total per expert.
+//   2. scatter: each block sums the segment totals of the whole grid (all S,
+//               for counts; those before it, for its own base) straight from
+//               L2, scans counts into offsets (block 0 writes counts and
+//               offsets), adds the per-warp histograms of the earlier warps of
+//               its segment, then every warp walks its sub-segment again in
+//               order, ranks each slot among its peers with the same id
 //               (popcount of lower lanes in the match mask) and writes
 //               sorted_token and dest_pos.
-// The workspace is seg: S x E int32, S = ceil(T*k_max / SEG).
+// Workspace: seg_total [S][E] and warp_hist [S][8][E], int32.
 #include <atomic>
 
 #include "common.cuh"
@@ -29,86 +31,118 @@ namespace {
 
 constexpr int kDispWarps = 8;
 constexpr int kMaxE = 512;
+constexpr int kBatch = 4;  // slot loads issued together per lane (items is a multiple)
+constexpr int kSumUnroll = 16;  // independent segment-total loads in flight per thread
 
-int seg_items(int64_t n_flat) {
+int warp_items(int64_t n_flat) {
     int items = 4;
-    while (n_flat > (int64_t)items * 32 * 1024 && items < 64) items *= 2;
+    while ((int64_t)items * 32 * kDispWarps * 148 < n_flat && items < 64) items *= 2;
     return items;
 }
 
-int64_t num_segments(int64_t n_flat, int items) { return (n_flat + items * 32 - 1) / (items * 32); }
+int64_t num_segments(int64_t n_flat, int items) {
+    const int64_t seg = (int64_t)items * 32 * kDispWarps;
+    return (n_flat + seg - 1) / seg;
+}
+
+__device__ __forceinline__ int load_id(const int32_t *ids, int64_t a, int64_t n_flat, int E,
+                                       bool &bad) {
+    int e = a < n_flat ? ids[a] : -1;
+    if (e < -1 || e >= E) {
+        bad = true;
+        e = -1;
+    }
+    return e;
+}
 
 __global__ void __launch_bounds__(kDispWarps * 32)
     dispatch_count_kernel(const int32_t *__restrict__ ids, int64_t n_flat, int E, int items,
-                          int64_t S, int32_t *__restrict__ seg, int32_t *status) {
+                          int32_t *__restrict__ seg_total, int32_t *__restrict__ warp_hist,
+                          int32_t *status) {
     __shared__ int32_t hist[kDispWarps][kMaxE];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t s = (int64_t)blockIdx.x * kDispWarps + warp;
-    if (s >= S) return;  // whole warp leaves together
-    int32_t *h = hist[warp];
-    for (int e = lane; e < E; e += 32) h[e] = 0;
+    const int64_t s = blockIdx.x;
+    for (int e = lane; e < E; e += 32) hist[warp][e] = 0;
     __syncwarp();
-    const int64_t base = s * items * 32;
+    const int64_t base = (s * kDispWarps + warp) * (int64_t)items * 32;
     bool bad = false;
-    for (int i = 0; i < items; ++i) {
-        const int64_t a = base + (int64_t)i * 32 + lane;
-        int e = a < n_flat ? ids[a] : -1;
-        if (e < -1 || e >= E) {
-            bad = true;
-            e = -1;
+    for (int i0 = 0; i0 < items; i0 += kBatch) {
+        int eb[kBatch];  // loads of a batch are issued before any of them is used
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j)
+            eb[j] = load_id(ids, base + (int64_t)(i0 + j) * 32 + lane, n_flat, E, bad);
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+            const int e = eb[j];
+            const unsigned peers = __match_any_sync(MOE_FULL_MASK, e);
+            if (e >= 0 && lane == __ffs(peers) - 1) hist[warp][e] += __popc(peers);
+            __syncwarp();
         }
-        const unsigned peers = __match_any_sync(MOE_FULL_MASK, e);
-        if (e >= 0 && lane == __ffs(peers) - 1) h[e] += __popc(peers);
-        __syncwarp();
     }
     if (__any_sync(MOE_FULL_MASK, bad) && lane == 0) report(status, MOE_ERR_DEVICE_INDEX);
-    int32_t *out = seg + s * E;
-    for (int e = lane; e < E; e += 32) out[e] = h[e];
-}
-
-// Block b handles experts 32b .. 32b+31 (lane = expert), warp w a contiguous
-// chunk of segments.
-__global__ void __launch_bounds__(1024)
-    dispatch_scan_kernel(int32_t *__restrict__ seg, int64_t S, int E, int32_t *__restrict__ counts) {
-    __shared__ int32_t part[32][33];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int e = blockIdx.x * 32 + lane;
-    const int64_t chunk = (S + 31) / 32;
-    const int64_t s0 = warp * chunk;
-    const int64_t s1 = s0 + chunk < S ? s0 + chunk : S;
-    int32_t sum = 0;
-    if (e < E)
-        for (int64_t s = s0; s < s1; ++s) sum += seg[s * E + e];
-    part[warp][lane] = sum;
+    int32_t *wh = warp_hist + (s * kDispWarps + warp) * E;
+    for (int e = lane; e < E; e += 32) wh[e] = hist[warp][e];
     __syncthreads();
-    int32_t run = 0;
-    for (int w = 0; w < warp; ++w) run += part[w][lane];
-    if (e < E) {
-        for (int64_t s = s0; s < s1; ++s) {
-            const int32_t v = seg[s * E + e];
-            seg[s * E + e] = run;
-            run += v;
-        }
-        if (warp == 31) counts[e] = run;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int32_t t = 0;
+#pragma unroll
+        for (int w = 0; w < kDispWarps; ++w) t += hist[w][e];
+        seg_total[s * E + e] = t;
     }
 }
 
 __global__ void __launch_bounds__(kDispWarps * 32)
     dispatch_scatter_kernel(const int32_t *__restrict__ ids, int64_t n_flat, int k_max, int E,
-                            int items, int64_t S, const int32_t *__restrict__ seg,
-                            const int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
-                            int32_t *__restrict__ sorted_token, int32_t *__restrict__ dest_pos) {
-    __shared__ int32_t off[kMaxE + 1];
+                            int items, int64_t S, const int32_t *__restrict__ seg_total,
+                            const int32_t *__restrict__ warp_hist, int32_t *__restrict__ counts,
+                            int32_t *__restrict__ offsets, int32_t *__restrict__ sorted_token,
+                            int32_t *__restrict__ dest_pos) {
+    __shared__ int32_t total[kMaxE + 1];
+    __shared__ int32_t before[kMaxE];
     __shared__ int32_t run[kDispWarps][kMaxE];
     __shared__ int32_t wsum[kDispWarps];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t s = blockIdx.x;
 
-    // Block-wide exclusive scan of counts: thread i owns experts 2i, 2i+1.
+    // Per-expert totals over all segments and over the segments before this one.
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        total[e] = 0;
+        before[e] = 0;
+    }
+    __syncthreads();
+    // Lane = expert within a 32-wide chunk, warp = every 8th segment: each
+    // load is a coalesced 128-byte line, and kSumUnroll of them are in flight
+    // per thread before any is added.
+    for (int c = 0; c < E; c += 32) {
+        const int e = c + lane;
+        int32_t acc_t = 0, acc_b = 0;
+        for (int64_t sp0 = warp; sp0 < S; sp0 += (int64_t)kDispWarps * kSumUnroll) {
+            int32_t v[kSumUnroll];
+#pragma unroll
+            for (int u = 0; u < kSumUnroll; ++u) {
+                const int64_t sp = sp0 + (int64_t)u * kDispWarps;
+                v[u] = (e < E && sp < S) ? seg_total[sp * E + e] : 0;
+            }
+#pragma unroll
+            for (int u = 0; u < kSumUnroll; ++u) {
+                acc_t += v[u];
+                acc_b += (sp0 + (int64_t)u * kDispWarps < s) ? v[u] : 0;
+            }
+        }
+        if (e < E) {
+            atomicAdd(&total[e], acc_t);
+            atomicAdd(&before[e], acc_b);
+        }
+    }
+    __syncthreads();
+
+    // Exclusive scan of the totals into offsets: thread i owns experts 2i, 2i+1.
     {
         const int i0 = 2 * threadIdx.x, i1 = i0 + 1;
-        const int32_t c0 = i0 < E ? counts[i0] : 0;
-        const int32_t c1 = i1 < E ? counts[i1] : 0;
-        int32_t v = c0 + c1, incl = v;
+        const int32_t c0 = i0 < E ? total[i0] : 0;
+        const int32_t c1 = i1 < E ? total[i1] : 0;
+        const int32_t v = c0 + c1;
+        int32_t incl = v;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int32_t n = __shfl_up_sync(MOE_FULL_MASK, incl, o);
@@ -116,44 +150,68 @@ __global__ void __launch_bounds__(kDispWarps * 32)
         }
         if (lane == 31) wsum[warp] = incl;
         __syncthreads();
-        int32_t before = 0;
-        for (int w = 0; w < warp; ++w) before += wsum[w];
-        const int32_t excl = before + incl - v;
-        if (i0 < E) off[i0] = excl;
-        if (i1 < E) off[i1] = excl + c0;
-        if (threadIdx.x == 0) {
-            int32_t total = 0;
-            for (int w = 0; w < kDispWarps; ++w) total += wsum[w];
-            off[E] = total;
+        int32_t pre = 0;
+        for (int w = 0; w < warp; ++w) pre += wsum[w];
+        const int32_t excl = pre + incl - v;
+        if (blockIdx.x == 0) {
+            if (i0 < E) {
+                counts[i0] = c0;
+                offsets[i0] = excl;
+            }
+            if (i1 < E) {
+                counts[i1] = c1;
+                offsets[i1] = excl + c0;
+            }
+            if (threadIdx.x == 0) {
+                int32_t all = 0;
+                for (int w = 0; w < kDispWarps; ++w) all += wsum[w];
+                offsets[E] = all;
+            }
         }
+        // Each warp's starting position per expert: offset + earlier segments +
+        // earlier warps of this segment.
         __syncthreads();
-        if (blockIdx.x == 0)
-            for (int e = threadIdx.x; e <= E; e += blockDim.x) offsets[e] = off[e];
+        if (i0 < E) total[i0] = excl;
+        if (i1 < E) total[i1] = excl + c0;
+        __syncthreads();
     }
-
-    const int64_t s = (int64_t)blockIdx.x * kDispWarps + warp;
-    if (s >= S) return;
+    const int32_t *wh = warp_hist + s * kDispWarps * E;
     int32_t *r = run[warp];
-    const int32_t *sb = seg + s * E;
-    for (int e = lane; e < E; e += 32) r[e] = off[e] + sb[e];
+    for (int e = lane; e < E; e += 32) {
+        int32_t v[kDispWarps];
+#pragma unroll
+        for (int w = 0; w < kDispWarps; ++w) v[w] = w < warp ? wh[w * E + e] : 0;
+        int32_t b = total[e] + before[e];
+#pragma unroll
+        for (int w = 0; w < kDispWarps; ++w) b += v[w];
+        r[e] = b;
+    }
     __syncwarp();
-    const int64_t base = s * items * 32;
+
+    const int64_t base = (s * kDispWarps + warp) * (int64_t)items * 32;
     const unsigned lower = (1u << lane) - 1u;
-    for (int i = 0; i < items; ++i) {
-        const int64_t a = base + (int64_t)i * 32 + lane;
-        int e = a < n_flat ? ids[a] : -1;
-        if (e < -1 || e >= E) e = -1;
-        const unsigned peers = __match_any_sync(MOE_FULL_MASK, e);
-        if (e >= 0) {
-            const int32_t pos = r[e] + __popc(peers & lower);
-            sorted_token[pos] = (int32_t)(a / k_max);
-            dest_pos[a] = pos;
-        } else if (a < n_flat) {
-            dest_pos[a] = -1;
+    bool bad = false;
+    for (int i0 = 0; i0 < items; i0 += kBatch) {
+        int eb[kBatch];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j)
+            eb[j] = load_id(ids, base + (int64_t)(i0 + j) * 32 + lane, n_flat, E, bad);
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+            const int64_t a = base + (int64_t)(i0 + j) * 32 + lane;
+            const int e = eb[j];
+            const unsigned peers = __match_any_sync(MOE_FULL_MASK, e);
+            if (e >= 0) {
+                const int32_t pos = r[e] + __popc(peers & lower);
+                sorted_token[pos] = (int32_t)(a / k_max);
+                dest_pos[a] = pos;
+            } else if (a < n_flat) {
+                dest_pos[a] = -1;
+            }
+            __syncwarp();
+            if (e >= 0 && lane == __ffs(peers) - 1) r[e] += __popc(peers);
+            __syncwarp();
         }
-        __syncwarp();
-        if (e >= 0 && lane == __ffs(peers) - 1) r[e] += __popc(peers);
-        __syncwarp();
     }
 }
 
@@ -167,8 +225,8 @@ extern "C" moe_status moe_dispatch_workspace_size(int64_t T, int32_t k_max, int3
         return MOE_ERR_INVALID_ARG;
     const int64_t n_flat = T * (int64_t)k_max;
     if (n_flat >= (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
-    const int64_t S = num_segments(n_flat, seg_items(n_flat));
-    const size_t b = (size_t)S * (size_t)E * sizeof(int32_t);
+    const int64_t S = num_segments(n_flat, warp_items(n_flat));
+    const size_t b = (size_t)S * (size_t)E * sizeof(int32_t) * (1 + kDispWarps);
     *bytes = (b + 255) / 256 * 256;
     return MOE_OK;
 }
@@ -188,18 +246,19 @@ extern "C" moe_status moe_dispatch(const int32_t *topk_ids, int64_t T, int32_t k
     if (n_flat > 0 && ((reinterpret_cast<uintptr_t>(workspace) & 255u) || ws_bytes < need))
         return MOE_ERR_INVALID_ARG;
     cudaStream_t cs = as_cuda(stream);
-    const int items = seg_items(n_flat);
+    const int items = warp_items(n_flat);
     const int64_t S = num_segments(n_flat, items);
-    int32_t *seg = static_cast<int32_t *>(workspace);
     if (S > 0) {
-        const unsigned blocks = (unsigned)((S + kDispWarps - 1) / kDispWarps);
-        dispatch_count_kernel<<<blocks, kDispWarps * 32, 0, cs>>>(topk_ids, n_flat, E, items, S,
-                                                                  seg, d_status);
-        dispatch_scan_kernel<<<(E + 31) / 32, 1024, 0, cs>>>(seg, S, E, counts);
-        dispatch_scatter_kernel<<<blocks, kDispWarps * 32, 0, cs>>>(
-            topk_ids, n_flat, k_max, E, items, S, seg, counts, offsets, sorted_token, dest_pos);
+        int32_t *seg_total = static_cast<int32_t *>(workspace);
+        int32_t *warp_hist = seg_total + S * E;
+        dispatch_count_kernel<<<(unsigned)S, kDispWarps * 32, 0, cs>>>(topk_ids, n_flat, E, items,
+                                                                      seg_total, warp_hist,
+                                                                      d_status);
+        dispatch_scatter_kernel<<<(unsigned)S, kDispWarps * 32, 0, cs>>>(
+            topk_ids, n_flat, k_max, E, items, S, seg_total, warp_hist, counts, offsets,
+            sorted_token, dest_pos);
     } else {
-        // No slots: every count is 0 and every offset is 0.
+        // No slots: every count and every offset is 0.
         if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, cs) != cudaSuccess ||
             cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), cs) != cudaSuccess) {
             cudaGetLastError();

@@ -9,14 +9,28 @@
 //   largest keys (equal keys -> lower id); weight = unbiased score, optionally
 //   renormalised, times route_scale.
 //
-// B200 design: a row of E <= 512 fp32 logits is spread over the 32 lanes of a
-// warp (128-bit loads when E % 4 == 0: lane l holds experts 128c + 4l .. +3 of
-// chunk c).  Selection keys are order-preserving uint32 images of the fp32
-// keys, so a round of top-k is two single-instruction warp reductions
-// (redux.sync max over keys, min over the ids that hold the max).  When no
-// bias is given and the group score is an amax, every score function is
-// monotone in the logit, so selection runs on the raw logits and only the k
-// selected experts are ever scored.
+// B200 design.
+//  * Memory: the kernel is persistent; each block streams tiles of R logits
+//    rows (contiguous in memory) into a ring of shared-memory stages with 1-D
+//    TMA bulk copies (cp.async.bulk, completion on an mbarrier), so several
+//    tiles per SM are in flight while warps compute on an earlier one.
+//  * Layout: a row of E <= 512 keys is spread over the 32 lanes of a warp;
+//    when E % 4 == 0 lane l holds experts 128c + 4l .. 128c + 4l + 3 of chunk
+//    c (128-bit shared loads), otherwise experts 32s + l.
+//  * Keys: a selection key is one 64-bit word, hi = order-preserving image of
+//    the fp32 key (larger float -> larger word, -0 == +0, NaN below every
+//    number, 0 = not selectable), lo = 511 - expert id.  Every word is
+//    distinct, a larger word is a better expert, and equal keys rank the lower
+//    id first, so selection is exact.  Each lane sorts its words once
+//    (Batcher's odd-even merge network); a top-k round is then two warp
+//    reductions (redux.sync max of hi, then max of lo among the lanes holding
+//    that hi) and a register shift in the one lane that owned the winner.
+//  * Monotone shortcut: with no bias and an amax group score, every score
+//    function orders experts like their logits, so keys are the logits and
+//    only the selected experts are ever scored.
+//  * Groups: when groups align with the 4-expert lane vectors and the 128-wide
+//    chunks, a group's top-2 is merged with register shuffles; otherwise each
+//    lane scans a strip of the group in shared memory.
 #include "common.cuh"
 
 namespace moe {
@@ -24,6 +38,8 @@ namespace {
 
 constexpr int kRouteWarps = 8;  // warps per block
 constexpr int kMaxE = 512;
+constexpr int kStages = 3;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 struct RouteArgs {
     const float *logits;
@@ -35,16 +51,77 @@ struct RouteArgs {
     int64_t T;
     int E, k_max, score, G, TG, topn, renorm;
     float scale;
-    int gsz, lpg, strip;      // group size, lanes per group, experts per lane strip
+    int gsz;                  // group size E / G
+    int lpg, strip;           // shared-memory group path: lanes per group, strip length
+    int group_mode;           // 0 none, 1 shuffle (gsz <= 128), 2 shuffle (gsz multiple of 128), 3 smem
     int keys_from_scores;     // 0: select on the logit (monotone case)
+    int R;                    // rows per tile (multiple of 8)
+    int64_t ntiles;
+    int red_width;            // power of two >= k_max (width of the weight reductions)
 };
+
+// ---------------------------------------------------------------- helpers --
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t *status) {
+    if (mbar_try(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try(bar, parity)) return true;
+        if ((it & 255u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) {
+            report(status, MOE_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// Copies `bytes` (a multiple of 16, may be 0) from global src to shared dst;
+// completion is counted on the mbarrier's transaction count.
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+    if (bytes)
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                dst),
+            "l"(src), "r"(bytes), "r"(bar)
+            : "memory");
+}
 
 template <bool VEC>
 __device__ __forceinline__ int slot_expert(int s, int lane) {
     return VEC ? (s >> 2) * 128 + lane * 4 + (s & 3) : s * 32 + lane;
 }
 
-// Keep the two largest finite-or-infinite values seen (NaN never enters).
+// Order-preserving image of an fp32 key: larger float -> larger word; -0 and
+// +0 equal; NaN -> 1 (below -inf, whose image is 0x007fffff); 0 is reserved.
+__device__ __forceinline__ uint32_t key_bits(float v) {
+    uint32_t u = __float_as_uint(v);
+    u = (v == 0.0f) ? 0u : u;
+    const uint32_t o = u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);
+    return (v != v) ? 1u : o;
+}
+
+// Keep the two largest values seen (NaN never enters).
 __device__ __forceinline__ void top2_insert(float v, float &t1, float &t2) {
     if (v > t1) {
         t2 = t1;
@@ -54,207 +131,467 @@ __device__ __forceinline__ void top2_insert(float v, float &t1, float &t2) {
     }
 }
 
+__device__ __forceinline__ void top2_merge(float &t1, float &t2, float b1, float b2) {
+    const float n1 = fmaxf(t1, b1);
+    const float n2 = fmaxf(fminf(t1, b1), fmaxf(t2, b2));
+    t1 = n1;
+    t2 = n2;
+}
+
+// Width-limited butterfly reductions (lanes >= width contribute the identity).
+__device__ __forceinline__ float sum_width(float v, int width) {
+    for (int o = 1; o < width; o <<= 1) v += __shfl_xor_sync(MOE_FULL_MASK, v, o);
+    return v;
+}
+__device__ __forceinline__ float max_width(float v, int width) {
+    for (int o = 1; o < width; o <<= 1) v = fmaxf(v, __shfl_xor_sync(MOE_FULL_MASK, v, o));
+    return v;
+}
+
+// Descending compare-exchange on (hi, lo) words.
+__device__ __forceinline__ void cas_desc(uint32_t &ah, uint32_t &al, uint32_t &bh, uint32_t &bl) {
+    const bool swap = (bh > ah) || (bh == ah && bl > al);
+    const uint32_t th = swap ? bh : ah, tl = swap ? bl : al;
+    bh = swap ? ah : bh;
+    bl = swap ? al : bl;
+    ah = th;
+    al = tl;
+}
+
+// Comparators of Batcher's odd-even merge sort of N (power of two) elements,
+// listed at compile time so that every register index is a constant.
+struct Comparators {
+    int n;
+    int a[80];
+    int b[80];
+};
+
+__host__ __device__ constexpr Comparators batcher(int N) {
+    Comparators c{};
+    for (int p = 1; p < N; p <<= 1)
+        for (int k = p; k >= 1; k >>= 1)
+            for (int j = k % p; j + k < N; j += 2 * k)
+                for (int i = 0; i < k; ++i)
+                    if (i + j + k < N && (i + j) / (2 * p) == (i + j + k) / (2 * p)) {
+                        c.a[c.n] = i + j;
+                        c.b[c.n] = i + j + k;
+                        ++c.n;
+                    }
+    return c;
+}
+
+// Sorts N (power of two) words in descending order.
+template <int N>
+__device__ __forceinline__ void sort_desc(uint32_t (&h)[N], uint32_t (&l)[N]) {
+    constexpr Comparators net = batcher(N);
+#pragma unroll
+    for (int c = 0; c < net.n; ++c) cas_desc(h[net.a[c]], l[net.a[c]], h[net.b[c]], l[net.b[c]]);
+}
+
+template <int V>
+struct Pow2 {
+    static constexpr int value = V <= 1 ? 1 : V <= 2 ? 2 : V <= 4 ? 4 : V <= 8 ? 8 : 16;
+};
+
 template <bool VEC, int VPL>
-__global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const RouteArgs a) {
-    __shared__ float sh_keys[kRouteWarps][kMaxE];
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int E = a.E;
-
-    // Per-lane constants: which expert each slot holds, its group, its bias.
-    int eid[VPL];
-    int gidx[VPL];
-    float biasr[VPL];
+__device__ __forceinline__ void load_row(const float *src, int lane, int E, float (&l)[VPL]) {
+    if (VEC) {
 #pragma unroll
-    for (int s = 0; s < VPL; ++s) {
-        int e = slot_expert<VEC>(s, lane);
-        eid[s] = e < E ? e : -1;
-        gidx[s] = (e < E && a.G > 1) ? e / a.gsz : 0;
-        biasr[s] = (a.bias && e < E) ? a.bias[e] : 0.0f;
-    }
-    const int my_g = lane / a.lpg;
-    const int my_p = lane % a.lpg;
-
-    for (int64_t row = (int64_t)blockIdx.x * kRouteWarps + warp; row < a.T;
-         row += (int64_t)gridDim.x * kRouteWarps) {
-        const float *lrow = a.logits + row * E;
-        float l[VPL];
-        if (VEC) {
-#pragma unroll
-            for (int c = 0; c < VPL / 4; ++c) {
-                const int e0 = c * 128 + lane * 4;
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (e0 < E) v = ld_stream(reinterpret_cast<const float4 *>(lrow + e0));
-                l[4 * c + 0] = v.x;
-                l[4 * c + 1] = v.y;
-                l[4 * c + 2] = v.z;
-                l[4 * c + 3] = v.w;
-            }
-        } else {
-#pragma unroll
-            for (int s = 0; s < VPL; ++s) l[s] = eid[s] >= 0 ? ld_stream(lrow + eid[s]) : 0.0f;
+        for (int c = 0; c < VPL / 4; ++c) {
+            const int e0 = c * 128 + lane * 4;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (e0 < E) v = *reinterpret_cast<const float4 *>(src + e0);
+            l[4 * c + 0] = v.x;
+            l[4 * c + 1] = v.y;
+            l[4 * c + 2] = v.z;
+            l[4 * c + 3] = v.w;
         }
-
-        int kt = a.k_max;
-        if (a.kpt) {
-            kt = a.kpt[row];
-            if (kt < 0 || kt > a.k_max) {
-                if (lane == 0) report(a.status, MOE_ERR_DEVICE_INDEX);
-                kt = kt < 0 ? 0 : a.k_max;
-            }
-        }
-
-        bool has_nan = false;
-#pragma unroll
-        for (int s = 0; s < VPL; ++s) has_nan |= (eid[s] >= 0) && (l[s] != l[s]);
-        if (__any_sync(MOE_FULL_MASK, has_nan) && lane == 0) report(a.status, MOE_ERR_NAN_LOGIT);
-
-        // Softmax statistics of the whole row, only when a weight or a key
-        // needs the full-row denominator.
-        float m = -INFINITY, z = 1.0f;
-        const bool need_z =
-            a.score == MOE_SCORE_SOFTMAX && (a.keys_from_scores || !a.renorm);
-        if (need_z) {
-            float lm = -INFINITY;
-#pragma unroll
-            for (int s = 0; s < VPL; ++s)
-                if (eid[s] >= 0) lm = fmaxf(lm, l[s]);
-            m = warp_max(lm);
-            float ls = 0.0f;
-#pragma unroll
-            for (int s = 0; s < VPL; ++s)
-                if (eid[s] >= 0) ls += expf(l[s] - m);
-            z = warp_sum(ls);
-        }
-
-        // Selection keys.
-        uint32_t key[VPL];
-        float *kb = sh_keys[warp];
+    } else {
 #pragma unroll
         for (int s = 0; s < VPL; ++s) {
-            float v = l[s];
-            if (a.keys_from_scores) {
-                if (a.score == MOE_SCORE_SOFTMAX)
-                    v = expf(l[s] - m) / z;
-                else if (a.score == MOE_SCORE_SIGMOID)
-                    v = sigmoid_score(l[s]);
-                else if (a.score == MOE_SCORE_SQRT_SOFTPLUS)
-                    v = sqrt_softplus_score(l[s]);
-                v += biasr[s];
-            }
-            key[s] = eid[s] >= 0 ? order_key(v) : 0u;
-            if (a.G > 1 && eid[s] >= 0) kb[eid[s]] = v;
-        }
-
-        // Group limit: per-group top-n sum over a lane strip, merged across
-        // the lanes of the group, then topk_groups rounds of warp argmax.
-        if (a.G > 1) {
-            __syncwarp();
-            float t1 = -INFINITY, t2 = -INFINITY;
-            if (my_g < a.G) {
-                const int lo = my_g * a.gsz + my_p * a.strip;
-                const int hi = min(lo + a.strip, (my_g + 1) * a.gsz);
-                for (int e = lo; e < hi; ++e) top2_insert(kb[e], t1, t2);
-            }
-            for (int o = 1; o < a.lpg; o <<= 1) {
-                const float b1 = __shfl_xor_sync(MOE_FULL_MASK, t1, o);
-                const float b2 = __shfl_xor_sync(MOE_FULL_MASK, t2, o);
-                const float n1 = fmaxf(t1, b1);
-                const float n2 = fmaxf(fminf(t1, b1), fmaxf(t2, b2));
-                t1 = n1;
-                t2 = n2;
-            }
-            __syncwarp();
-            const float gs = a.topn == 1 ? t1 : t1 + t2;
-            uint32_t gk = (my_g < a.G && my_p == 0) ? order_key(gs) : 0u;
-            uint32_t kept = 0;
-            for (int r = 0; r < a.TG; ++r) {
-                const uint32_t mx = __reduce_max_sync(MOE_FULL_MASK, gk);
-                const uint32_t cand = (gk == mx) ? (uint32_t)my_g : 0xffffffffu;
-                const uint32_t win = __reduce_min_sync(MOE_FULL_MASK, cand);
-                kept |= 1u << win;
-                if ((uint32_t)my_g == win) gk = 0u;
-            }
-#pragma unroll
-            for (int s = 0; s < VPL; ++s)
-                if (!((kept >> gidx[s]) & 1u)) key[s] = 0u;
-        }
-
-        // Top-k_t: each round takes the largest key, lowest id among equals.
-        uint32_t bk = 0u;
-        int bid = 0x7fffffff;
-#pragma unroll
-        for (int s = 0; s < VPL; ++s)
-            if (key[s] > bk) {
-                bk = key[s];
-                bid = eid[s];
-            }
-        int my_id = -1;
-        float my_l = 0.0f;
-        int nsel = 0;
-        for (int r = 0; r < kt; ++r) {
-            const uint32_t mx = __reduce_max_sync(MOE_FULL_MASK, bk);
-            if (mx == 0u) break;
-            const uint32_t cand = (bk == mx) ? (uint32_t)bid : 0xffffffffu;
-            const int win = (int)__reduce_min_sync(MOE_FULL_MASK, cand);
-            const int owner = VEC ? ((win & 127) >> 2) : (win & 31);
-            float lw = 0.0f;
-            if (lane == owner) {
-                bk = 0u;
-                bid = 0x7fffffff;
-#pragma unroll
-                for (int s = 0; s < VPL; ++s) {
-                    if (eid[s] == win) {
-                        lw = l[s];
-                        key[s] = 0u;
-                    }
-                    if (key[s] > bk) {
-                        bk = key[s];
-                        bid = eid[s];
-                    }
-                }
-            }
-            lw = __shfl_sync(MOE_FULL_MASK, lw, owner);
-            if (lane == r) {
-                my_id = win;
-                my_l = lw;
-            }
-            ++nsel;
-        }
-
-        // Weights of the selected experts, one per lane.
-        const bool act = lane < nsel;
-        float s = 0.0f;
-        if (a.score == MOE_SCORE_SOFTMAX && !a.renorm) {
-            s = act ? expf(my_l - m) / z : 0.0f;
-        } else if (a.score == MOE_SCORE_SOFTMAX || a.score == MOE_SCORE_TOPK_SOFTMAX) {
-            const float msel = warp_max(act ? my_l : -INFINITY);
-            s = act ? expf(my_l - msel) : 0.0f;
-        } else if (a.score == MOE_SCORE_SIGMOID) {
-            s = act ? sigmoid_score(my_l) : 0.0f;
-        } else {
-            s = act ? sqrt_softplus_score(my_l) : 0.0f;
-        }
-        if (a.renorm || a.score == MOE_SCORE_TOPK_SOFTMAX) {
-            const float sum = warp_sum(s);
-            if (act && sum > 0.0f) s = s / sum;
-        }
-        if (lane < a.k_max) {
-            a.ids[row * a.k_max + lane] = act ? my_id : -1;
-            a.w[row * a.k_max + lane] = act ? s * a.scale : 0.0f;
+            const int e = s * 32 + lane;
+            l[s] = e < E ? src[e] : 0.0f;
         }
     }
 }
 
-template <bool VEC>
-cudaError_t launch_route(const RouteArgs &a, int vpl, dim3 grid, cudaStream_t st) {
-    switch (vpl) {
-        case 4: route_kernel<VEC, 4><<<grid, kRouteWarps * 32, 0, st>>>(a); break;
-        case 8: route_kernel<VEC, 8><<<grid, kRouteWarps * 32, 0, st>>>(a); break;
-        case 12: route_kernel<VEC, 12><<<grid, kRouteWarps * 32, 0, st>>>(a); break;
-        default: route_kernel<VEC, 16><<<grid, kRouteWarps * 32, 0, st>>>(a); break;
+// One token row: keys, group limit, top-k_t, weights, stores.
+template <bool VEC, int VPL>
+__device__ __forceinline__ void route_row(const RouteArgs &a, const float *src, int kt,
+                                          int64_t row, int lane, const float (&biasr)[VPL],
+                                          const int (&gidx)[VPL], float *kscratch) {
+    constexpr int NP = Pow2<VPL>::value;
+    const int E = a.E;
+    float l[VPL];
+    load_row<VEC, VPL>(src, lane, E, l);
+
+    if (kt < 0 || kt > a.k_max) {
+        if (lane == 0) report(a.status, MOE_ERR_DEVICE_INDEX);
+        kt = kt < 0 ? 0 : a.k_max;
     }
-    return cudaSuccess;
+
+    bool has_nan = false;
+#pragma unroll
+    for (int s = 0; s < VPL; ++s) has_nan |= (slot_expert<VEC>(s, lane) < E) && (l[s] != l[s]);
+    if (__any_sync(MOE_FULL_MASK, has_nan) && lane == 0) report(a.status, MOE_ERR_NAN_LOGIT);
+
+    // Full-row softmax statistics, only where a key or a weight needs them.
+    float m = -INFINITY, z = 1.0f;
+    if (a.score == MOE_SCORE_SOFTMAX && (a.keys_from_scores || !a.renorm)) {
+        float lm = -INFINITY;
+#pragma unroll
+        for (int s = 0; s < VPL; ++s)
+            if (slot_expert<VEC>(s, lane) < E) lm = fmaxf(lm, l[s]);
+        m = warp_max(lm);
+        float ls = 0.0f;
+#pragma unroll
+        for (int s = 0; s < VPL; ++s)
+            if (slot_expert<VEC>(s, lane) < E) ls += expf(l[s] - m);
+        z = warp_sum(ls);
+    }
+
+    // Selection keys as fp32 values.
+    float v[VPL];
+    if (a.keys_from_scores) {
+        const float zinv = 1.0f / z;
+#pragma unroll
+        for (int s = 0; s < VPL; ++s) {
+            float x = l[s];
+            if (a.score == MOE_SCORE_SOFTMAX)
+                x = expf(l[s] - m) * zinv;
+            else if (a.score == MOE_SCORE_SIGMOID)
+                x = __frcp_rn(1.0f + expf(-l[s]));
+            else if (a.score == MOE_SCORE_SQRT_SOFTPLUS)
+                x = sqrt_softplus_score(l[s]);
+            v[s] = x + biasr[s];
+        }
+    } else {
+#pragma unroll
+        for (int s = 0; s < VPL; ++s) v[s] = l[s];
+    }
+
+    // Group limit -> bit mask of kept groups.
+    uint32_t kept = 0xffffffffu;
+    if (a.group_mode != 0) {
+        float my_gs = -INFINITY;
+        if (a.group_mode == 1) {
+            const int lg = a.gsz >> 2;     // lanes per group within a chunk
+            const int gpc = 128 / a.gsz;   // groups per chunk
+#pragma unroll
+            for (int c = 0; c < VPL / 4; ++c) {
+                float t1 = -INFINITY, t2 = -INFINITY;
+                if (c * 128 + lane * 4 < E)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) top2_insert(v[4 * c + j], t1, t2);
+                for (int o = 1; o < lg; o <<= 1) {
+                    const float b1 = __shfl_xor_sync(MOE_FULL_MASK, t1, o);
+                    const float b2 = __shfl_xor_sync(MOE_FULL_MASK, t2, o);
+                    top2_merge(t1, t2, b1, b2);
+                }
+                const float gs = a.topn == 1 ? t1 : t1 + t2;
+                const float got = __shfl_sync(MOE_FULL_MASK, gs, (lane % gpc) * lg);
+                if (lane / gpc == c) my_gs = got;
+            }
+        } else if (a.group_mode == 2) {
+            const int cpg = a.gsz / 128;  // chunks per group
+#pragma unroll
+            for (int g = 0; g < VPL / 4; ++g) {
+                if (g >= a.G) break;
+                float t1 = -INFINITY, t2 = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < VPL / 4; ++c)
+                    if (c / cpg == g && c * 128 + lane * 4 < E)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) top2_insert(v[4 * c + j], t1, t2);
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float b1 = __shfl_xor_sync(MOE_FULL_MASK, t1, o);
+                    const float b2 = __shfl_xor_sync(MOE_FULL_MASK, t2, o);
+                    top2_merge(t1, t2, b1, b2);
+                }
+                if (lane == g) my_gs = a.topn == 1 ? t1 : t1 + t2;
+            }
+        } else {
+            // Strip scan in shared memory: lane (g, p) takes part p of group g.
+#pragma unroll
+            for (int s = 0; s < VPL; ++s) {
+                const int e = slot_expert<VEC>(s, lane);
+                if (e < E) kscratch[e] = v[s];
+            }
+            __syncwarp();
+            const int g = lane / a.lpg, p = lane % a.lpg;
+            float t1 = -INFINITY, t2 = -INFINITY;
+            if (g < a.G) {
+                const int lo = g * a.gsz + p * a.strip;
+                const int hi = min(lo + a.strip, (g + 1) * a.gsz);
+                for (int e = lo; e < hi; ++e) top2_insert(kscratch[e], t1, t2);
+            }
+            for (int o = 1; o < a.lpg; o <<= 1) {
+                const float b1 = __shfl_xor_sync(MOE_FULL_MASK, t1, o);
+                const float b2 = __shfl_xor_sync(MOE_FULL_MASK, t2, o);
+                top2_merge(t1, t2, b1, b2);
+            }
+            __syncwarp();
+            const float gs = a.topn == 1 ? t1 : t1 + t2;
+            const float got = __shfl_sync(MOE_FULL_MASK, gs, (lane < a.G ? lane : 0) * a.lpg);
+            my_gs = got;
+        }
+        uint32_t gk = lane < a.G ? key_bits(my_gs) : 0u;
+        if (lane < a.G && gk == 0u) gk = 1u;
+        kept = 0u;
+        for (int r = 0; r < a.TG; ++r) {
+            const uint32_t mx = __reduce_max_sync(MOE_FULL_MASK, gk);
+            const uint32_t cand = (gk == mx) ? (uint32_t)lane : 32u;
+            const uint32_t win = __reduce_min_sync(MOE_FULL_MASK, cand);
+            kept |= 1u << win;
+            if ((uint32_t)lane == win) gk = 0u;
+        }
+    }
+
+    // 64-bit selection words, sorted per lane.
+    uint32_t kh[NP], kl[NP];
+#pragma unroll
+    for (int s = 0; s < NP; ++s) {
+        kh[s] = 0u;
+        kl[s] = 0u;
+    }
+#pragma unroll
+    for (int s = 0; s < VPL; ++s) {
+        const int e = slot_expert<VEC>(s, lane);
+        const bool ok = e < E && ((kept >> gidx[s]) & 1u);
+        kh[s] = ok ? key_bits(v[s]) : 0u;
+        kl[s] = ok ? (uint32_t)(511 - e) : 0u;
+    }
+    sort_desc<NP>(kh, kl);
+
+    // Top-k_t rounds.
+    uint32_t sel_lo = 0u;
+    int nsel = 0;
+    for (; nsel < kt; ++nsel) {
+        const uint32_t mh = __reduce_max_sync(MOE_FULL_MASK, kh[0]);
+        if (mh == 0u) break;
+        const bool hit = kh[0] == mh;
+        const uint32_t ml = __reduce_max_sync(MOE_FULL_MASK, hit ? kl[0] : 0u);
+        const bool pop = hit && kl[0] == ml;
+#pragma unroll
+        for (int i = 0; i + 1 < NP; ++i) {
+            kh[i] = pop ? kh[i + 1] : kh[i];
+            kl[i] = pop ? kl[i + 1] : kl[i];
+        }
+        kh[NP - 1] = pop ? 0u : kh[NP - 1];
+        kl[NP - 1] = pop ? 0u : kl[NP - 1];
+        if (lane == nsel) sel_lo = ml;
+    }
+
+    // Weights of the selected experts, one per lane.
+    const bool act = lane < nsel;
+    const int my_id = 511 - (int)sel_lo;
+    const float my_l = act ? src[my_id] : 0.0f;
+    float s = 0.0f;
+    if (a.score == MOE_SCORE_SOFTMAX && !a.renorm) {
+        s = act ? expf(my_l - m) / z : 0.0f;
+    } else if (a.score == MOE_SCORE_SOFTMAX || a.score == MOE_SCORE_TOPK_SOFTMAX) {
+        const float msel = max_width(act ? my_l : -INFINITY, a.red_width);
+        s = act ? expf(my_l - msel) : 0.0f;
+    } else if (a.score == MOE_SCORE_SIGMOID) {
+        s = act ? sigmoid_score(my_l) : 0.0f;
+    } else {
+        s = act ? sqrt_softplus_score(my_l) : 0.0f;
+    }
+    if (a.renorm || a.score == MOE_SCORE_TOPK_SOFTMAX) {
+        const float sum = sum_width(s, a.red_width);
+        if (act && sum > 0.0f) s = s / sum;
+    }
+    if (lane < a.k_max) {
+        a.ids[row * a.k_max + lane] = act ? my_id : -1;
+        a.w[row * a.k_max + lane] = act ? s * a.scale : 0.0f;
+    }
+}
+
+// k_max == 1 without groups: the argmax of the keys (lowest id among equal
+// keys) and its weight; no per-lane sort and a single warp round.
+template <bool VEC, int VPL>
+__device__ __forceinline__ void route_row_top1(const RouteArgs &a, const float *src, int kt,
+                                               int64_t row, int lane, const float (&biasr)[VPL]) {
+    const int E = a.E;
+    float l[VPL];
+    load_row<VEC, VPL>(src, lane, E, l);
+    if (kt < 0 || kt > 1) {
+        if (lane == 0) report(a.status, MOE_ERR_DEVICE_INDEX);
+        kt = kt < 0 ? 0 : 1;
+    }
+    float m = -INFINITY, z = 1.0f;
+    bool has_nan = false;
+#pragma unroll
+    for (int s = 0; s < VPL; ++s)
+        if (slot_expert<VEC>(s, lane) < E) {
+            has_nan |= l[s] != l[s];
+            m = fmaxf(m, l[s]);
+        }
+    if (__any_sync(MOE_FULL_MASK, has_nan) && lane == 0) report(a.status, MOE_ERR_NAN_LOGIT);
+    if (a.score == MOE_SCORE_SOFTMAX && (a.keys_from_scores || !a.renorm)) {
+        m = warp_max(m);
+        float ls = 0.0f;
+#pragma unroll
+        for (int s = 0; s < VPL; ++s)
+            if (slot_expert<VEC>(s, lane) < E) ls += expf(l[s] - m);
+        z = warp_sum(ls);
+    }
+    // Lane's best key (the first slot wins ties: slots ascend in expert id).
+    uint32_t bk = 0u;
+    int be = 0x7fffffff;
+    const float zinv = 1.0f / z;
+#pragma unroll
+    for (int s = 0; s < VPL; ++s) {
+        const int e = slot_expert<VEC>(s, lane);
+        float v = l[s];
+        if (a.keys_from_scores) {
+            if (a.score == MOE_SCORE_SOFTMAX)
+                v = expf(l[s] - m) * zinv;
+            else if (a.score == MOE_SCORE_SIGMOID)
+                v = __frcp_rn(1.0f + expf(-l[s]));
+            else if (a.score == MOE_SCORE_SQRT_SOFTPLUS)
+                v = sqrt_softplus_score(l[s]);
+            v += biasr[s];
+        }
+        const uint32_t k = e < E ? key_bits(v) : 0u;
+        if (k > bk) {
+            bk = k;
+            be = e;
+        }
+    }
+    const uint32_t mx = __reduce_max_sync(MOE_FULL_MASK, bk);
+    const int win = (int)__reduce_min_sync(MOE_FULL_MASK, bk == mx ? (uint32_t)be : 0xffffffffu);
+    if (lane == 0) {
+        const bool act = kt == 1 && mx != 0u;
+        float s = 0.0f;
+        if (act) {
+            const float lw = src[win];
+            if (a.score == MOE_SCORE_SOFTMAX && !a.renorm)
+                s = expf(lw - m) / z;
+            else if (a.score == MOE_SCORE_SOFTMAX || a.score == MOE_SCORE_TOPK_SOFTMAX)
+                s = 1.0f;  // softmax over the single selected expert
+            else if (a.score == MOE_SCORE_SIGMOID)
+                s = sigmoid_score(lw);
+            else
+                s = sqrt_softplus_score(lw);
+            if (a.renorm && s > 0.0f) s = s / s;
+        }
+        a.ids[row] = act ? win : -1;
+        a.w[row] = act ? s * a.scale : 0.0f;
+    }
+}
+
+template <bool VEC, int VPL, bool TOP1>
+__global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const RouteArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int E = a.E;
+    const int R = a.R;
+    const size_t stage_floats = (size_t)R * E;
+    // [stages x R x E logits][stages x R k_per_token][stages mbarriers]
+    float *stages = reinterpret_cast<float *>(smem);
+    int32_t *kstages = reinterpret_cast<int32_t *>(stages + kStages * stage_floats);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(kstages + kStages * R);
+    float *kscratch = reinterpret_cast<float *>(bars + kStages) + (size_t)warp * kMaxE;
+    // Per-lane constants: group of each slot, bias of each slot.
+    int gidx[VPL];
+    float biasr[VPL];
+#pragma unroll
+    for (int s = 0; s < VPL; ++s) {
+        const int e = slot_expert<VEC>(s, lane);
+        gidx[s] = (e < E && a.G > 1) ? e / a.gsz : 0;
+        biasr[s] = (a.bias && e < E) ? a.bias[e] : 0.0f;
+    }
+
+    auto tile_rows = [&](int64_t t) -> int {
+        const int64_t r0 = t * R;
+        return (int)(a.T - r0 < R ? a.T - r0 : R);
+    };
+    // Bytes of a tile that one bulk copy can carry (a multiple of 16).
+    auto tile_bytes = [&](int64_t t) -> uint32_t {
+        return (uint32_t)(((uint64_t)tile_rows(t) * E * sizeof(float)) & ~uint64_t(15));
+    };
+    // Bytes of the tile's k_per_token that one bulk copy can carry.
+    auto kpt_bytes = [&](int64_t t) -> uint32_t {
+        return a.kpt ? (uint32_t)(((uint32_t)tile_rows(t) * sizeof(int32_t)) & ~15u) : 0u;
+    };
+    auto issue = [&](int64_t t, int stage) {
+        const uint32_t bar = smem_u32(&bars[stage]);
+        const uint32_t lb = tile_bytes(t), kb = kpt_bytes(t);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+                     "r"(lb + kb)
+                     : "memory");
+        bulk_copy(smem_u32(stages + stage * stage_floats), a.logits + t * R * (int64_t)E, lb, bar);
+        bulk_copy(smem_u32(kstages + stage * R), a.kpt + t * R, kb, bar);
+    };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[s])) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (int s = 0; s < kStages; ++s) {
+            const int64_t t = blockIdx.x + (int64_t)s * gridDim.x;
+            if (t < a.ntiles) issue(t, s);
+        }
+    }
+    __syncthreads();
+
+    const int rpw = R / kRouteWarps;
+    int it = 0;
+    for (int64_t t = blockIdx.x; t < a.ntiles; t += gridDim.x, ++it) {
+        const int stage = it % kStages;
+        const bool ok = mbar_wait(smem_u32(&bars[stage]), (uint32_t)(it / kStages) & 1u, a.status);
+        if (!__syncthreads_and(ok)) break;
+        const int rows = tile_rows(t);
+        const int covered = (int)(tile_bytes(t) / ((uint32_t)E * sizeof(float)));
+        const int kcovered = (int)(kpt_bytes(t) / sizeof(int32_t));
+        const float *tile = stages + stage * stage_floats;
+        const int32_t *ktile = kstages + stage * R;
+        for (int i = 0; i < rpw; ++i) {
+            const int r = warp * rpw + i;
+            if (r >= rows) break;
+            const int64_t row = t * R + r;
+            const int kt = !a.kpt ? a.k_max : (r < kcovered ? ktile[r] : a.kpt[row]);
+            const float *src = r < covered ? tile + (size_t)r * E : a.logits + row * E;
+            if (TOP1)
+                route_row_top1<VEC, VPL>(a, src, kt, row, lane, biasr);
+            else
+                route_row<VEC, VPL>(a, src, kt, row, lane, biasr, gidx, kscratch);
+        }
+        __syncthreads();  // every warp is done with this stage
+        if (threadIdx.x == 0) {
+            const int64_t nt = t + (int64_t)kStages * gridDim.x;
+            if (nt < a.ntiles) issue(nt, stage);
+        }
+    }
+    // A wait that timed out leaves later tiles unconsumed: let their copies land.
+    if (threadIdx.x == 0) {
+        for (int64_t t = blockIdx.x + (int64_t)it * gridDim.x, j = it;
+             t < a.ntiles && j < it + kStages; t += gridDim.x, ++j)
+            if (!mbar_wait(smem_u32(&bars[j % kStages]), (uint32_t)(j / kStages) & 1u, a.status))
+                break;
+    }
+}
+
+template <bool VEC>
+void *route_fn(int vpl, bool top1) {
+    if (top1) {
+        switch (vpl) {
+            case 4: return (void *)route_kernel<VEC, 4, true>;
+            case 8: return (void *)route_kernel<VEC, 8, true>;
+            case 12: return (void *)route_kernel<VEC, 12, true>;
+            default: return (void *)route_kernel<VEC, 16, true>;
+        }
+    }
+    switch (vpl) {
+        case 4: return (void *)route_kernel<VEC, 4, false>;
+        case 8: return (void *)route_kernel<VEC, 8, false>;
+        case 12: return (void *)route_kernel<VEC, 12, false>;
+        default: return (void *)route_kernel<VEC, 16, false>;
+    }
 }
 
 // ------------------------------------------------------------- hash route --
@@ -345,7 +682,9 @@ extern "C" moe_status moe_route(const float *logits, const float *bias, const in
                   p->group_topn > 2 || p->group_topn > E / G || p->k_max > p->topk_groups * (E / G)))
         return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
-    if (!logits || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
+    if (!logits || !topk_ids || !topk_w || !aligned16(logits) ||
+        (k_per_token && !aligned16(k_per_token)))
+        return MOE_ERR_INVALID_ARG;
     if (T > (int64_t)INT32_MAX / (p->k_max > 0 ? p->k_max : 1)) return MOE_ERR_UNSUPPORTED;
 
     RouteArgs a;
@@ -370,18 +709,50 @@ extern "C" moe_status moe_route(const float *logits, const float *bias, const in
     a.lpg = lpg;
     a.strip = (a.gsz + lpg - 1) / lpg;
     a.keys_from_scores = (bias != nullptr) || (G > 1 && a.topn > 1);
+    const bool vec = (E % 4 == 0);
+    if (G == 1)
+        a.group_mode = 0;
+    else if (vec && a.gsz % 4 == 0 && 128 % a.gsz == 0)
+        a.group_mode = 1;
+    else if (vec && a.gsz % 128 == 0)
+        a.group_mode = 2;
+    else
+        a.group_mode = 3;
+    int R = (4096 / E) / 8 * 8;
+    R = R < 8 ? 8 : (R > 256 ? 256 : R);
+    a.R = R;
+    a.ntiles = (T + R - 1) / R;
+    int width = 1;
+    while (width < p->k_max) width *= 2;
+    a.red_width = width;
 
-    const bool vec = (E % 4 == 0) && aligned16(logits);
     const int vpl_need = vec ? 4 * ((E + 127) / 128) : (E + 31) / 32;
     const int vpl = vpl_need <= 4 ? 4 : vpl_need <= 8 ? 8 : vpl_need <= 12 ? 12 : 16;
-    const int64_t blocks_needed = (T + kRouteWarps - 1) / kRouteWarps;
-    const int64_t cap = (int64_t)sm_count() * 8;
-    dim3 grid((unsigned)(blocks_needed < cap ? blocks_needed : cap));
-    cudaStream_t st = as_cuda(stream);
-    if (vec)
-        launch_route<true>(a, vpl, grid, st);
-    else
-        launch_route<false>(a, vpl, grid, st);
+    const bool top1 = p->k_max == 1 && G == 1;
+    void *fn = vec ? route_fn<true>(vpl, top1) : route_fn<false>(vpl, top1);
+    const size_t smem = (size_t)kStages * R * E * sizeof(float) + (size_t)kStages * R * sizeof(int32_t) +
+                        kStages * sizeof(uint64_t) +
+                        (a.group_mode == 3 ? (size_t)kRouteWarps * kMaxE * sizeof(float) : 0);
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kRouteWarps * 32, smem) !=
+            cudaSuccess ||
+        per_sm < 1) {
+        cudaGetLastError();
+        per_sm = 1;
+    }
+    const int64_t cap = (int64_t)sm_count() * per_sm;
+    const unsigned grid = (unsigned)(a.ntiles < cap ? a.ntiles : cap);
+    void *args[] = {&a};
+    if (cudaLaunchKernel(fn, dim3(grid), dim3(kRouteWarps * 32), args, smem, as_cuda(stream)) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
     return launch_status();
 }
 
