@@ -115,26 +115,27 @@ def load_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(files) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "token_dispatch_moe_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in files:
         with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(workload: str, kernel: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on the
-    current kernel sources; else None."""
+    kernel's current source files; else None."""
     try:
         with open(TRAFFIC_FILE) as f:
             rec = json.load(f)
-    except (OSError, ValueError):
+        entry = rec["workloads"][workload][kernel]
+    except (OSError, ValueError, KeyError):
         return None
-    if rec.get("source_hash") != kernel_source_hash():
+    if entry.get("sha") != kernel_source_hash(entry.get("files", [])):
         return None
-    return rec.get("workloads", {}).get(workload, {}).get(kernel)
+    return entry.get("bytes")
 
 
 # --------------------------------------------------------------------- clocks

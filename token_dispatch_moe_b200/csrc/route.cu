@@ -718,7 +718,13 @@ extern "C" moe_status moe_route(const float *logits, const float *bias, const in
         a.group_mode = 2;
     else
         a.group_mode = 3;
+    // Rows per tile: about 16 KB of logits, but small enough that every SM
+    // gets at least two tiles (each row is a serial chain of warp reductions,
+    // so small batches need the rows spread out).
+    const int sms = sm_count();
     int R = (4096 / E) / 8 * 8;
+    const int64_t spread = ((T + 2 * sms - 1) / (2 * sms) + 7) / 8 * 8;
+    if (spread < R) R = (int)spread;
     R = R < 8 ? 8 : (R > 256 ? 256 : R);
     a.R = R;
     a.ntiles = (T + R - 1) / R;
@@ -745,7 +751,7 @@ extern "C" moe_status moe_route(const float *logits, const float *bias, const in
         cudaGetLastError();
         per_sm = 1;
     }
-    const int64_t cap = (int64_t)sm_count() * per_sm;
+    const int64_t cap = (int64_t)sms * per_sm;
     const unsigned grid = (unsigned)(a.ntiles < cap ? a.ntiles : cap);
     void *args[] = {&a};
     if (cudaLaunchKernel(fn, dim3(grid), dim3(kRouteWarps * 32), args, smem, as_cuda(stream)) !=
