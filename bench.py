@@ -90,16 +90,26 @@ def rank_seed_offset(rank: int) -> int:
 
 
 # ------------------------------------------------------------------ byte model
-def stage_bytes(wl, n_assign: int) -> dict:
+def stage_bytes(wl, n_assign: int, fused: bool = False, limited=None) -> dict:
     """Algorithmic DRAM bytes per launch of each kernel (each read once, each
-    write once) and the gate's FLOPs."""
+    write once) and the gate's FLOPs.  limited = (kept slots, tokens with a
+    kept slot, padding rows) of a capacity-limited dispatch: only kept slots
+    move rows, only tokens with one are read, padding rows cost a 4-byte -1."""
     T, d, E, k = wl.T, wl.d, wl.E, wl.k_max
+    t_read, pad_rows = T, 0
+    if limited is not None:
+        n_assign, t_read, pad_rows = limited
     b = {}
-    if wl.gate:
-        b["gate_gemm"] = T * d * 2 + E * d * 2 + T * E * 4
-    b["route"] = T * E * 4 + T * k * 8 + (T * 4 if wl.k_choices else 0) + (E * 4 if wl.bias else 0)
-    b["dispatch"] = T * k * 4 + n_assign * 4 + T * k * 4 + 8 * E
-    b["permute"] = T * d * 2 + n_assign * d * 2 + T * k * 4
+    if wl.gate and fused:
+        b["gate_route"] = (T * d * 2 + E * d * 2 + T * k * 8 + (T * 4 if wl.k_choices else 0)
+                           + (E * 4 if wl.bias else 0))
+    else:
+        if wl.gate:
+            b["gate_gemm"] = T * d * 2 + E * d * 2 + T * E * 4
+        b["route"] = (T * E * 4 + T * k * 8 + (T * 4 if wl.k_choices else 0)
+                      + (E * 4 if wl.bias else 0))
+    b["dispatch"] = T * k * 4 + n_assign * 4 + T * k * 4 + 8 * E + pad_rows * 4
+    b["permute"] = t_read * d * 2 + n_assign * d * 2 + T * k * 4
     if wl.combine:
         b["combine"] = n_assign * d * 2 + T * d * 2 + (T * d * 2 if wl.shared else 0) + 8 * T * k
     return b
@@ -209,6 +219,7 @@ def oracle_inputs(wl, inp: dict, n_tokens: int) -> dict:
     kpt = inp["k_per_token"]
     h["kpt"] = kpt[:n_tokens].cpu().numpy() if kpt is not None else None
     n = int(h["kpt"].sum()) if kpt is not None else n_tokens * wl.k_max
+    n += wl.E * (wl.pad - 1)  # padded expert blocks
     h["y"] = bits(normal_bf16((max(n, 1), wl.d), 1.0, "cpu", 1000 * wl.index + 44))
     h["shared"] = bits(inp["shared"][:n_tokens]) if inp["shared"] is not None else None
     return h
@@ -224,7 +235,11 @@ def oracle_chain(wl, h: dict) -> None:
     r = oracle.route(logits, k_max=wl.k_max, score=score, bias=h["bias"], k_per_token=h["kpt"],
                      n_groups=wl.n_groups, topk_groups=wl.topk_groups, group_topn=wl.group_topn,
                      renormalize=wl.renormalize, route_scale=wl.route_scale)
-    dsp = oracle.dispatch(r["ids"], wl.E)
+    if wl.limited:  # the same capacity rule, applied to the sample's own tokens
+        dsp = oracle.dispatch_limited(r["ids"], wl.E, capacity=wl.scaled(h["T"]).capacity,
+                                      pad=wl.pad)
+    else:
+        dsp = oracle.dispatch(r["ids"], wl.E)
     n = int(dsp["offsets"][-1])
     oracle.permute(h["x"], dsp["dest_pos"], n)
     if wl.combine:
@@ -243,9 +258,10 @@ def oracle_sample_size(wl, inp, budget_s: float) -> int:
 
 
 # ----------------------------------------------------------------- our arm
-def chain_launches(wl) -> int:
+def chain_launches(wl, fused: bool) -> int:
     """Kernels of this library launched by one step of the chain."""
-    return (1 if wl.gate else 0) + 1 + 3 + 1 + (1 if wl.combine else 0)
+    gate_route = 1 if fused else (1 if wl.gate else 0) + 1
+    return gate_route + 2 + 1 + (1 if wl.combine else 0)
 
 
 def run_ours(args):
@@ -263,11 +279,11 @@ def run_ours(args):
         wl = wl.scaled(args.tokens)
     inp = make_inputs(wl, device, seed_offset=rank_seed_offset(rank))
     n_assign = num_assignments(wl, inp["k_per_token"])
-    path = RouterDispatch(wl, device)
+    path = RouterDispatch(wl, device, fused=False if args.separate else (True if args.fused else None))
     stream = torch.cuda.current_stream(device)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=device)
-    bytes_per = stage_bytes(wl, n_assign)
+    bytes_per = stage_bytes(wl, n_assign, path.fused)
     names = list(bytes_per)
 
     def run_step(mark):
@@ -281,12 +297,16 @@ def run_ours(args):
             i += 1
 
         boundary()
-        logits = inp["logits"]
-        if wl.gate:
-            logits = path.gate(inp["x"], inp["w"])
+        if path.fused:
+            path.gate_route(inp["x"], inp["w"], inp["bias"], inp["k_per_token"])
             boundary()
-        path.route(logits, inp["bias"], inp["k_per_token"])
-        boundary()
+        else:
+            logits = inp["logits"]
+            if wl.gate:
+                logits = path.gate(inp["x"], inp["w"])
+                boundary()
+            path.route(logits, inp["bias"], inp["k_per_token"])
+            boundary()
         path.dispatch()
         boundary()
         path.permute(inp["x"])
@@ -301,6 +321,12 @@ def run_ours(args):
     torch.cuda.synchronize()
     if path.status.item() != 0:
         raise RuntimeError(f"device status {moe.moe_status_string(path.status.item())}")
+    limited = None
+    if wl.limited:  # what the capacity kept decides the bytes moved
+        kept = n_assign - path.dropped.item()
+        t_read = int((path.dest_pos >= 0).any(dim=1).sum().item())
+        limited = (kept, t_read, int(path.offsets[-1].item()) - kept)
+        bytes_per = stage_bytes(wl, n_assign, path.fused, limited)
 
     K = args.steps
     nb = len(names) + 1
@@ -373,10 +399,11 @@ def run_ours(args):
         gbs = bytes_per[n] / (stage_ms[n] / 1e3) / 1e9
         stages[n] = {"us": round(stage_ms[n] * 1e3, 2), "bytes": bytes_per[n],
                      "GB_s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4)}
+    gname = "gate_route" if path.fused else "gate_gemm"
     if wl.gate:
         flops = 2.0 * wl.T * wl.E * wl.d
-        stages["gate_gemm"]["TFLOP_s"] = round(flops / (stage_ms["gate_gemm"] / 1e3) / 1e12, 1)
-        stages["gate_gemm"]["frac_tensor"] = round(stages["gate_gemm"]["TFLOP_s"] / tf_sust, 4)
+        stages[gname]["TFLOP_s"] = round(flops / (stage_ms[gname] / 1e3) / 1e12, 1)
+        stages[gname]["frac_tensor"] = round(stages[gname]["TFLOP_s"] / tf_sust, 4)
     dom = max(stage_ms, key=stage_ms.get)
     achieved = bytes_per[dom] / (stage_ms[dom] / 1e3) / 1e9
     roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
@@ -401,9 +428,13 @@ def run_ours(args):
                    "inputs": "bf16 x / W / expert outputs, fp32 logits",
                    "l2": f"flushed before every timed step ({flush.numel() * 4 >> 20} MiB write)",
                    "parallelism": f"token-sharded replicas x{world}",
-                   "launch": "stream (eager)" if args.eager else "CUDA graph of the step"},
+                   "launch": "stream (eager)" if args.eager else "CUDA graph of the step",
+                   "gate_route": "fused (one kernel)" if path.fused else "separate kernels",
+                   **({"capacity": path.capacity, "capacity_factor": wl.capacity_factor,
+                       "pad_rows_to": wl.pad, "kept_slots": limited[0],
+                       "dropped_slots": n_assign - limited[0]} if limited else {})},
         "roofline": roofline, "stages": stages, "clocks": clk.summary(),
-        "gpu_launches": chain_launches(wl) * K, "e2e": e2e,
+        "gpu_launches": chain_launches(wl, path.fused) * K, "e2e": e2e,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl, inp, args.cpu_budget)
@@ -504,6 +535,10 @@ def main(argv=None):
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the workload's token count (profiling of smaller cases)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--separate", action="store_true",
+                    help="run the gate GEMM and the route as two kernels instead of one")
+    ap.add_argument("--fused", action="store_true",
+                    help="route inside the gate GEMM even where two kernels are faster")
     ap.add_argument("--eager", action="store_true",
                     help="launch from the host every step instead of replaying a CUDA graph")
     ap.add_argument("--no-e2e", action="store_true")

@@ -130,6 +130,21 @@ moe_status moe_route(const float *logits, const float *bias, const int32_t *k_pe
                      float *topk_w, int32_t *d_status, moe_stream_t stream);
 
 /*
+ * moe_gate_route -- moe_gate_gemm and moe_route in one kernel (the gate linear
+ * and the router are one function in "DeepSeek-V3.2-Exp - Select experts",
+ * gate forward).  Same inputs, outputs and status rules as the two calls in a
+ * row, except that the logits are written only if `logits` is non-NULL: each
+ * token's row of logits is routed straight from the tensor-core accumulator.
+ * Selected ids are the same as moe_route's on the same logits; weights agree
+ * to rounding.  Limits: k_max <= 16 (else MOE_ERR_UNSUPPORTED), plus those of
+ * both calls.
+ */
+moe_status moe_gate_route(const moe_bf16_t *x, const moe_bf16_t *w, const float *bias,
+                          const int32_t *k_per_token, const moe_route_params *params, int64_t T,
+                          int32_t d, int32_t *topk_ids, float *topk_w, float *logits,
+                          int32_t *d_status, moe_stream_t stream);
+
+/*
  * moe_hash_route -- expert ids from a token-id table ("Crate ferrox_moe",
  * route_hash: the DeepSeek-V4 hash layers look the ids up by token id; no
  * bias, no selection).
@@ -172,6 +187,43 @@ moe_status moe_dispatch(const int32_t *topk_ids, int64_t T, int32_t k_max, int32
                         int32_t *counts, int32_t *offsets, int32_t *sorted_token,
                         int32_t *dest_pos, void *workspace, size_t ws_bytes, int32_t *d_status,
                         moe_stream_t stream);
+
+/*
+ * moe_dispatch_limited_rows -- rows that sorted_token (and the permuted xs)
+ * must hold for moe_dispatch_limited with these sizes:
+ *   min(T*k_max, E*capacity) + E*(pad - 1)   (capacity 0: T*k_max + E*(pad-1)).
+ * capacity >= 0, 1 <= pad <= 4096; MOE_ERR_UNSUPPORTED when the bound reaches 2^31.
+ */
+moe_status moe_dispatch_limited_rows(int64_t T, int32_t k_max, int32_t E, int32_t capacity,
+                                     int32_t pad, int64_t *rows);
+
+/*
+ * moe_dispatch_limited -- moe_dispatch with a per-expert capacity and expert
+ * blocks padded for a tiled expert GEMM.  The capacity is the Switch-style
+ * top-1 limit the open-MoE router survey lists among the router levers ("I
+ * modelli MoE open hanno router opposti"); the pages give no formula, and the
+ * reading here is: expert e keeps the first `capacity` of its slots in flat
+ * order a = t*k_max + j and drops the others.  capacity 0 keeps every slot.
+ *   counts[e]   = number of slots with id e (the demand, before the cut);
+ *   kept[e]     = min(counts[e], capacity);
+ *   offsets[0]  = 0, offsets[e+1] = offsets[e] + kept[e] rounded up to a
+ *                 multiple of pad;
+ *   a kept slot of rank r (earlier slots with the same e) gets
+ *   pos = offsets[e] + r, sorted_token[pos] = t, dest_pos[a] = pos;
+ *   a dropped or empty slot gets dest_pos[a] = -1;
+ *   sorted_token[offsets[e] + kept[e] .. offsets[e+1]) = -1 (padding rows);
+ *   *dropped (nullable) = sum over e of counts[e] - kept[e].
+ * sorted_rows: capacity of sorted_token, >= moe_dispatch_limited_rows().
+ * capacity 0 with pad 1 gives exactly moe_dispatch's outputs.  moe_permute and
+ * moe_combine take the dest_pos as they are (dropped slots are skipped; the
+ * padding rows of xs are not written).  Workspace, alignment, device-error
+ * and stream rules as moe_dispatch.
+ */
+moe_status moe_dispatch_limited(const int32_t *topk_ids, int64_t T, int32_t k_max, int32_t E,
+                                int32_t capacity, int32_t pad, int32_t *counts, int32_t *offsets,
+                                int32_t *sorted_token, int64_t sorted_rows, int32_t *dest_pos,
+                                int32_t *dropped, void *workspace, size_t ws_bytes,
+                                int32_t *d_status, moe_stream_t stream);
 
 /*
  * moe_dispatch_static -- moe_dispatch without a caller-provided workspace.
@@ -220,6 +272,68 @@ moe_status moe_permute(const moe_bf16_t *x, const int32_t *dest_pos, int64_t T, 
 moe_status moe_combine(const moe_bf16_t *y, const float *topk_w, const int32_t *dest_pos,
                        const moe_bf16_t *shared, int64_t T, int32_t k_max, int32_t d,
                        moe_bf16_t *out, moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Expert-parallel exchange.  In multi-GPU expert parallelism every router
+ * choice becomes all-to-all traffic ("I modelli MoE open hanno router
+ * opposti", closing paragraphs); here that traffic is the permute's stores and
+ * the combine's loads themselves, made over peer memory (NVLink) with plain
+ * 16-byte accesses.  G ranks, expert e on rank e / (E/G).
+ * Receive layout of rank d (the pages fix none; this is the plain reading):
+ * its experts in ascending order; inside one expert the rows of source rank 0,
+ * then 1, ...; inside one source, that rank's slots in flat order.
+ * Per step on every rank: moe_dispatch (local) -> all-gather of counts ->
+ * moe_ep_layout -> moe_ep_permute -> barrier -> experts on the receive buffer
+ * -> barrier -> moe_ep_combine.  The all-gather and the barriers are the
+ * caller's collectives (e.g. NCCL); nothing here waits on another GPU.
+ * ------------------------------------------------------------------------ */
+
+/*
+ * moe_ep_layout -- owner rank and receive row of every slot of this rank.
+ *   all_counts [G][E]: every rank's moe_dispatch counts (gathered);
+ *   topk_ids, dest_pos [T][k_max], offsets [E+1]: this rank's moe_dispatch
+ *   inputs and outputs;
+ *   dest_rank[a] = e / (E/G);  dest_row[a] = row of slot a on that rank
+ *   (both -1 for an empty slot);
+ *   recv_offsets [E/G + 1]: this rank's receive blocks, recv_offsets[le] =
+ *   first row of its local expert le, recv_offsets[E/G] = rows it receives.
+ * 1 <= G <= 64, 0 <= rank < G, E <= 512, E % G == 0.  A slot whose dest_pos
+ * disagrees with offsets/all_counts, or an id outside [-1, E), gets -1/-1
+ * and reports MOE_ERR_DEVICE_INDEX.
+ */
+moe_status moe_ep_layout(const int32_t *all_counts, const int32_t *topk_ids,
+                         const int32_t *dest_pos, const int32_t *offsets, int32_t G, int32_t rank,
+                         int64_t T, int32_t k_max, int32_t E, int32_t *dest_rank,
+                         int32_t *dest_row, int32_t *recv_offsets, int32_t *d_status,
+                         moe_stream_t stream);
+
+/*
+ * moe_ep_permute -- recv_r[dest_row[t][j]] = x[t] with r = dest_rank[t][j]:
+ * each row of x is read once and stored to its owners' receive buffers.
+ * peer_recv: DEVICE array of G pointers, entry r = rank r's receive buffer
+ * ([recv_capacity][d] bf16, 16-byte aligned) as mapped in this process (its
+ * own buffer for r == this rank).  A (rank, row) outside [0,G) x
+ * [0,recv_capacity), or a null/unaligned entry, skips the slot and reports
+ * MOE_ERR_DEVICE_INDEX.  The receivers must not be using their buffers while
+ * this runs, and read them only after every sender's call has completed.
+ */
+moe_status moe_ep_permute(const moe_bf16_t *x, const int32_t *dest_rank, const int32_t *dest_row,
+                          moe_bf16_t *const *peer_recv, int32_t G, int64_t recv_capacity,
+                          int64_t T, int32_t k_max, int32_t d, int32_t *d_status,
+                          moe_stream_t stream);
+
+/*
+ * moe_ep_combine -- moe_combine whose expert rows live on their owners:
+ *   out[t] = bf16_rne( sum_j topk_w[t][j] * y_r[dest_row[t][j]] + shared[t] ),
+ *   r = dest_rank[t][j]; fp32 in slot order, shared added last.
+ * peer_y: DEVICE array of G pointers to the ranks' expert outputs
+ * ([recv_capacity][d] bf16, in receive layout).  Bounds and status as
+ * moe_ep_permute.  The owners' outputs must be complete before this runs.
+ */
+moe_status moe_ep_combine(moe_bf16_t *const *peer_y, const int32_t *dest_rank,
+                          const int32_t *dest_row, const float *topk_w, const moe_bf16_t *shared,
+                          int32_t G, int64_t recv_capacity, int64_t T, int32_t k_max, int32_t d,
+                          moe_bf16_t *out, int32_t *d_status, moe_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -78,6 +78,12 @@ def _bind(lib):
     lib.oracle_hash_route.restype = ctypes.c_int
     lib.oracle_dispatch.argtypes = [P, i64, i32, i32, P, P, P, P]
     lib.oracle_dispatch.restype = ctypes.c_int
+    lib.oracle_dispatch_limited.argtypes = [P, i64, i32, i32, i32, i32, P, P, P, P, P]
+    lib.oracle_dispatch_limited.restype = ctypes.c_int
+    lib.oracle_route_grouped.argtypes = [P, i64, i32, i32, i32, i32, i32, i32, f64, P, P, P]
+    lib.oracle_route_grouped.restype = ctypes.c_int
+    lib.oracle_ep_layout.argtypes = [P, i32, i64, i32, i32, P, P, P]
+    lib.oracle_ep_layout.restype = ctypes.c_int
     lib.oracle_permute.argtypes = [P, P, i64, i32, i32, P]
     lib.oracle_permute.restype = None
     lib.oracle_combine.argtypes = [P, P, P, P, i64, i32, i32, P, P]
@@ -156,6 +162,25 @@ def weights_for_ids(logits, ids, *, score, renormalize=True, route_scale=1.0) ->
     return w
 
 
+def route_grouped(logits, *, k_max, score, n_groups, k_per_group, renormalize=True,
+                  route_scale=1.0, want_keys=False):
+    """Grouped top-k (per-group k, then the global top k_max of the candidates)."""
+    lg = _c(logits, np.float32)
+    T, E = lg.shape
+    ids = np.empty((T, k_max), np.int32)
+    w = np.empty((T, k_max), np.float64)
+    keys = np.empty((T, E), np.float64) if want_keys else None
+    st = _load().oracle_route_grouped(_p(lg), T, E, k_max, score, n_groups, k_per_group,
+                                      int(renormalize), float(route_scale), _p(ids), _p(w),
+                                      _p(keys) if keys is not None else None)
+    if st == ERR_ARG:
+        raise ValueError("oracle_route_grouped: bad arguments")
+    out = {"ids": ids, "w": w, "status": st}
+    if want_keys:
+        out["keys"] = keys
+    return out
+
+
 def hash_route(tok, table, *, num_experts, logits=None, score=SOFTMAX, renormalize=True,
                route_scale=1.0):
     tok = _c(tok, np.int32)
@@ -182,6 +207,73 @@ def dispatch(ids, num_experts):
     n = int(offsets[-1])
     return {"counts": counts, "offsets": offsets, "sorted_token": sorted_token[:n],
             "dest_pos": dest_pos, "status": st}
+
+
+def dispatch_limited(ids, num_experts, capacity: int = 0, pad: int = 1):
+    """Dispatch with a per-expert capacity (0 = none) and expert blocks padded
+    to a multiple of ``pad`` rows; returns counts (demand), padded offsets,
+    sorted_token (padding rows -1), dest_pos (-1 for dropped slots), dropped."""
+    ids = _c(ids, np.int32)
+    T, k_max = ids.shape
+    counts = np.empty((num_experts,), np.int32)
+    offsets = np.empty((num_experts + 1,), np.int32)
+    rows = T * k_max if capacity <= 0 else min(T * k_max, num_experts * capacity)
+    rows += num_experts * (pad - 1)
+    sorted_token = np.full((max(rows, 1),), -7, np.int32)
+    dest_pos = np.empty((T, k_max), np.int32)
+    dropped = ctypes.c_int64(0)
+    st = _load().oracle_dispatch_limited(_p(ids), T, k_max, num_experts, capacity, pad,
+                                         _p(counts), _p(offsets), _p(sorted_token),
+                                         _p(dest_pos), ctypes.byref(dropped))
+    n = int(offsets[-1])
+    return {"counts": counts, "offsets": offsets, "sorted_token": sorted_token[:n],
+            "dest_pos": dest_pos, "dropped": int(dropped.value), "status": st}
+
+
+def ep_layout(ids_all, num_experts):
+    """Expert-parallel receive layout for G ranks' ids [G][T][k_max]: the owner
+    rank and row of every slot, and each rank's received row count."""
+    ids = _c(ids_all, np.int32)
+    G, T, k_max = ids.shape
+    dest_rank = np.empty((G, T, k_max), np.int32)
+    dest_row = np.empty((G, T, k_max), np.int32)
+    recv_rows = np.zeros((G,), np.int64)
+    st = _load().oracle_ep_layout(_p(ids), G, T, k_max, num_experts, _p(dest_rank), _p(dest_row),
+                                  _p(recv_rows))
+    return {"dest_rank": dest_rank, "dest_row": dest_row, "recv_rows": recv_rows, "status": st}
+
+
+def ep_permute(x_all_bits, dest_rank, dest_row, recv_rows):
+    """Each rank's receive buffer: recv[d][dest_row] = x[r][t] for every slot
+    (r, t, j) whose owner is d.  Rows are copied bit for bit."""
+    x = np.asarray(x_all_bits, np.uint16)
+    G, T, d = x.shape
+    recv = [np.zeros((int(recv_rows[g]), d), np.uint16) for g in range(G)]
+    for r in range(G):
+        for t in range(T):
+            for j in range(dest_rank.shape[2]):
+                g = dest_rank[r, t, j]
+                if g >= 0:
+                    recv[g][dest_row[r, t, j]] = x[r, t]
+    return recv
+
+
+def ep_combine(y_bits_per_rank, w_all, dest_rank, dest_row, shared_all_bits=None, want_mag=True):
+    """out[r][t] = sum_j w[r][t][j] * y[owner][row] (+ shared[r][t]): the
+    combine of one source rank reads each slot's row from its owner.  Built
+    from ``combine`` on the owners' rows laid end to end."""
+    G = dest_rank.shape[0]
+    starts = np.concatenate([[0], np.cumsum([y.shape[0] for y in y_bits_per_rank])])
+    y_cat = np.concatenate([np.asarray(y, np.uint16) for y in y_bits_per_rank], axis=0)
+    if y_cat.shape[0] == 0:
+        y_cat = np.zeros((1, y_bits_per_rank[0].shape[1]), np.uint16)
+    outs = []
+    for r in range(G):
+        gpos = np.where(dest_rank[r] >= 0, starts[np.maximum(dest_rank[r], 0)] + dest_row[r], -1)
+        outs.append(combine(y_cat, w_all[r], gpos.astype(np.int32),
+                            None if shared_all_bits is None else shared_all_bits[r],
+                            want_mag=want_mag))
+    return outs
 
 
 def permute(x_bits, dest_pos, n_rows: int) -> np.ndarray:

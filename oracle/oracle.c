@@ -262,6 +262,54 @@ int oracle_weights_for_ids(const float *logits, const int32_t *ids, int64_t T, i
     return ORACLE_OK;
 }
 
+/* ------------------------------------------------------- grouped route ---- */
+/* [FX] route_top_k_grouped: cut the E experts into n_groups contiguous groups,
+ * keep the k_per_group best of each group (by the same score as the flat
+ * router), then keep the total_k best of those candidates across groups.
+ * Readings: no bias (the page gives none for this rule); candidates and the
+ * final choice both rank by (score desc, id asc), the output in that order;
+ * total_k = k_max, the output width, and k_max <= n_groups * k_per_group;
+ * weights as the flat router (row_weights).  keys_out (optional) receives the
+ * candidates' scores and -inf for experts their group did not keep. */
+int oracle_route_grouped(const float *logits, int64_t T, int32_t E, int32_t k_max,
+                         int32_t score, int32_t n_groups, int32_t k_per_group,
+                         int32_t renormalize, double route_scale, int32_t *ids, double *w,
+                         double *keys_out) {
+    if (E <= 0 || n_groups < 1 || E % n_groups != 0 || k_per_group < 1 ||
+        k_per_group > E / n_groups || k_max < 0 || k_max > n_groups * k_per_group)
+        return ORACLE_ERR_ARG;
+    int status = ORACLE_OK;
+    const int32_t gsz = E / n_groups;
+    double *s = (double *)malloc(sizeof(double) * E);
+    ranked *grp = (ranked *)malloc(sizeof(ranked) * gsz);
+    ranked *cand = (ranked *)malloc(sizeof(ranked) * E);
+    for (int64_t t = 0; t < T; ++t) {
+        const float *l = logits + t * E;
+        row_scores(l, E, score, s);
+        int32_t nc = 0;
+        if (keys_out)
+            for (int32_t e = 0; e < E; ++e) keys_out[t * E + e] = -INFINITY;
+        for (int32_t g = 0; g < n_groups; ++g) {
+            for (int32_t i = 0; i < gsz; ++i) {
+                grp[i].key = s[g * gsz + i];
+                grp[i].id = g * gsz + i;
+                if (isnan(grp[i].key)) status = ORACLE_ERR_NAN;
+            }
+            qsort(grp, (size_t)gsz, sizeof(ranked), by_key_desc);
+            for (int32_t i = 0; i < k_per_group; ++i) {
+                cand[nc++] = grp[i];
+                if (keys_out) keys_out[t * E + grp[i].id] = grp[i].key;
+            }
+        }
+        qsort(cand, (size_t)nc, sizeof(ranked), by_key_desc);
+        int32_t *sel = ids + t * k_max;
+        for (int32_t j = 0; j < k_max; ++j) sel[j] = cand[j].id;
+        row_weights(l, s, sel, k_max, score, renormalize, route_scale, w + t * k_max);
+    }
+    free(s), free(grp), free(cand);
+    return status;
+}
+
 /* ---------------------------------------------------------- hash route ---- */
 /* [FX] route_hash: the expert ids of token t are row tok[t] of the table
  * (row-major [vocab][k], one row of k ids per token id; a repeated id in a row
@@ -340,6 +388,92 @@ int oracle_dispatch(const int32_t *ids, int64_t T, int32_t k_max, int32_t E, int
         }
     }
     free(seen);
+    return status;
+}
+
+/* ------------------------------------------- dispatch with a capacity ---- */
+/* Top-1 with a per-expert capacity in the Switch style (the open-MoE router
+ * survey, its paragraph on the five router levers) and expert blocks padded
+ * for a tiled expert GEMM.  Reading: expert e keeps the first `capacity` of its
+ * slots in flat order a = t*k_max + j and drops the rest (dest_pos = -1);
+ * capacity <= 0 keeps all.  Expert e's block holds kept[e] rows rounded up to
+ * a multiple of `pad`; offsets is the exclusive scan of the block sizes; the
+ * padding rows of sorted_token hold -1.  counts[e] is the demand before the
+ * capacity cut, *dropped the number of slots cut. */
+int oracle_dispatch_limited(const int32_t *ids, int64_t T, int32_t k_max, int32_t E,
+                            int32_t capacity, int32_t pad, int32_t *counts, int32_t *offsets,
+                            int32_t *sorted_token, int32_t *dest_pos, int64_t *dropped) {
+    int status = ORACLE_OK;
+    int64_t n = T * (int64_t)k_max;
+    for (int32_t e = 0; e < E; ++e) counts[e] = 0;
+    for (int64_t a = 0; a < n; ++a) {
+        int32_t e = ids[a];
+        if (e >= 0 && e < E)
+            counts[e] += 1;
+        else if (e != -1)
+            status = ORACLE_ERR_INDEX;
+    }
+    *dropped = 0;
+    offsets[0] = 0;
+    for (int32_t e = 0; e < E; ++e) {
+        int32_t kept = counts[e];
+        if (capacity > 0 && kept > capacity) {
+            *dropped += kept - capacity;
+            kept = capacity;
+        }
+        int32_t block = (kept + pad - 1) / pad * pad;
+        offsets[e + 1] = offsets[e] + block;
+        for (int32_t r = kept; r < block; ++r) sorted_token[offsets[e] + r] = -1;
+    }
+    int32_t *seen = (int32_t *)calloc((size_t)E, sizeof(int32_t));
+    for (int64_t a = 0; a < n; ++a) {
+        int32_t e = ids[a];
+        dest_pos[a] = -1;
+        if (e < 0 || e >= E) continue;
+        int32_t rank = seen[e];
+        seen[e] += 1;
+        if (capacity > 0 && rank >= capacity) continue;
+        int32_t pos = offsets[e] + rank;
+        sorted_token[pos] = (int32_t)(a / k_max);
+        dest_pos[a] = pos;
+    }
+    free(seen);
+    return status;
+}
+
+/* --------------------------------------------- expert-parallel exchange ---- */
+/* Expert-parallel placement (the open-MoE router survey: in multi-GPU expert
+ * parallelism every router choice becomes all-to-all traffic).  G ranks hold T
+ * tokens each; expert e lives on rank e / (E/G).  Reading of the receive
+ * layout: rank d's buffer holds its experts in ascending order; inside an
+ * expert, the rows of source rank 0, then rank 1, ...; inside a source, that
+ * rank's slots in flat order a = t*k_max + j.  ids_all is [G][T][k_max];
+ * dest_rank / dest_row [G][T][k_max] receive the owner rank and row of every
+ * slot (-1 / -1 for empty slots); recv_rows[d] the row count of rank d. */
+int oracle_ep_layout(const int32_t *ids_all, int32_t G, int64_t T, int32_t k_max, int32_t E,
+                     int32_t *dest_rank, int32_t *dest_row, int64_t *recv_rows) {
+    if (G < 1 || E % G != 0) return ORACLE_ERR_ARG;
+    int status = ORACLE_OK;
+    const int32_t el = E / G;
+    const int64_t n = T * (int64_t)k_max;
+    for (int64_t i = 0; i < (int64_t)G * n; ++i) {
+        dest_rank[i] = -1;
+        dest_row[i] = -1;
+        if (ids_all[i] < -1 || ids_all[i] >= E) status = ORACLE_ERR_INDEX;
+    }
+    for (int32_t d = 0; d < G; ++d) recv_rows[d] = 0;
+    /* Experts in ascending order visit the owners in order and each owner's
+     * experts in order; inside an expert, sources in rank order, then slots. */
+    for (int32_t e = 0; e < E; ++e) {
+        const int32_t d = e / el;
+        for (int32_t r = 0; r < G; ++r)
+            for (int64_t a = 0; a < n; ++a)
+                if (ids_all[(int64_t)r * n + a] == e) {
+                    dest_rank[(int64_t)r * n + a] = d;
+                    dest_row[(int64_t)r * n + a] = (int32_t)recv_rows[d];
+                    recv_rows[d] += 1;
+                }
+    }
     return status;
 }
 

@@ -268,6 +268,59 @@ def pin_weight_invariants():
     assert _rel_close(s1["w"][:, 0], 1.0 / (1.0 + np.exp(-lg.max(1).astype(np.float64))), 1e-14)
 
 
+def pin_route_grouped():
+    # Worked by hand: logits [5, 4, 3, 0, -1, -2], two groups of three, two
+    # candidates per group, keep 3.  Flat top-3 would be 0, 1, 2; the groups
+    # put expert 3 in place of 2.  Softmax weights over all six, renormalised
+    # over the three kept: e^5, e^4, e^0 over their sum.
+    lg = np.array([[5, 4, 3, 0, -1, -2]], np.float32)
+    r = oracle.route_grouped(lg, k_max=3, score=oracle.SOFTMAX, n_groups=2, k_per_group=2)
+    assert r["ids"].tolist() == [[0, 1, 3]]
+    z = math.exp(5) + math.exp(4) + 1.0
+    assert _rel_close(r["w"][0], np.array([math.exp(5) / z, math.exp(4) / z, 1.0 / z]), 1e-14)
+    flat = oracle.route(lg, k_max=3, score=oracle.SOFTMAX)
+    assert flat["ids"].tolist() == [[0, 1, 2]]
+    # Brute force in plain Python: per group sort by (-score, id), then again.
+    rng = np.random.default_rng(59)
+    scores = {oracle.SOFTMAX: None, oracle.SIGMOID: lambda v: 1.0 / (1.0 + math.exp(-v)),
+              oracle.SQRT_SOFTPLUS: lambda v: math.sqrt(max(v, 0.0) + math.log1p(math.exp(-abs(v)))),
+              oracle.TOPK_SOFTMAX: lambda v: v}
+    for E, G, kpg, k, sc, renorm, scale, integer in (
+            (16, 4, 2, 5, oracle.SOFTMAX, True, 1.0, False), (16, 4, 2, 8, oracle.SIGMOID, False, 2.0, True),
+            (24, 3, 3, 4, oracle.SQRT_SOFTPLUS, True, 1.5, False), (32, 8, 1, 8, oracle.TOPK_SOFTMAX, True, 1.0, True),
+            (12, 1, 5, 5, oracle.SIGMOID, True, 1.0, False), (20, 5, 4, 3, oracle.SOFTMAX, False, 1.0, True)):
+        lg = (rng.integers(-3, 4, size=(60, E)) if integer else rng.normal(size=(60, E))).astype(np.float32)
+        r = oracle.route_grouped(lg, k_max=k, score=sc, n_groups=G, k_per_group=kpg,
+                                 renormalize=renorm, route_scale=scale)
+        gsz = E // G
+        for t in range(lg.shape[0]):
+            row = [float(v) for v in lg[t]]
+            if sc == oracle.SOFTMAX:
+                m = max(row)
+                z = sum(math.exp(v - m) for v in row)
+                sv = [math.exp(v - m) / z for v in row]
+            else:
+                sv = [scores[sc](v) for v in row]
+            cand = []
+            for g in range(G):
+                members = sorted(range(g * gsz, (g + 1) * gsz), key=lambda e: (-sv[e], e))
+                cand += members[:kpg]
+            pick = sorted(cand, key=lambda e: (-sv[e], e))[:k]
+            assert r["ids"][t].tolist() == pick, (t, r["ids"][t], pick)
+            if sc == oracle.TOPK_SOFTMAX:
+                m = max(row[e] for e in pick)
+                ww = [math.exp(row[e] - m) for e in pick]
+            else:
+                ww = [sv[e] for e in pick]
+            if renorm:
+                tot = sum(ww)
+                ww = [v / tot for v in ww]
+            assert _rel_close(r["w"][t], np.array(ww) * scale, 1e-12)
+        if kpg == gsz or G == 1:  # every expert is a candidate: the flat router
+            f = oracle.route(lg, k_max=k, score=sc, renormalize=renorm, route_scale=scale)
+            assert np.array_equal(f["ids"], r["ids"])
+
+
 def pin_dynamic_k_prefix():
     """Per-token k picks a prefix of the same ranking; nothing else changes."""
     rng = np.random.default_rng(12)
@@ -380,6 +433,97 @@ def pin_dispatch_library():
     assert r["status"] == oracle.ERR_INDEX
 
 
+def pin_dispatch_limited():
+    # Worked by hand: six top-1 tokens on three experts, capacity 2, blocks
+    # padded to 4 rows.  Expert 0 is asked for by tokens 0, 2, 3, 5 and keeps
+    # the first two; experts 1 and 2 keep their one token each.
+    ids = np.array([[0], [1], [0], [0], [2], [0]], np.int32)
+    r = oracle.dispatch_limited(ids, 3, capacity=2, pad=4)
+    assert r["status"] == oracle.OK and r["dropped"] == 2
+    assert r["counts"].tolist() == [4, 1, 1]
+    assert r["offsets"].tolist() == [0, 4, 8, 12]
+    assert r["sorted_token"].tolist() == [0, 2, -1, -1, 1, -1, -1, -1, 4, -1, -1, -1]
+    assert r["dest_pos"].reshape(-1).tolist() == [0, 4, 1, -1, 8, -1]
+    # Brute force: each expert's kept slots are its first `cap` in flat order.
+    rng = np.random.default_rng(43)
+    for T, k_max, E, cap, pad in ((1, 1, 1, 0, 1), (40, 2, 5, 7, 1), (300, 4, 16, 50, 8),
+                                  (500, 8, 64, 0, 128), (257, 1, 8, 20, 16), (64, 6, 12, 1, 3)):
+        ids = rng.integers(0, E, size=(T, k_max)).astype(np.int32)
+        ids[rng.random(size=(T, k_max)) < 0.15] = -1
+        r = oracle.dispatch_limited(ids, E, capacity=cap, pad=pad)
+        flat = ids.reshape(-1)
+        dp = r["dest_pos"].reshape(-1)
+        st = r["sorted_token"]
+        base, dropped = 0, 0
+        for e in range(E):
+            slots = np.nonzero(flat == e)[0]
+            assert r["counts"][e] == slots.size
+            keep = slots if cap <= 0 else slots[:cap]
+            dropped += slots.size - keep.size
+            block = -(-keep.size // pad) * pad
+            assert r["offsets"][e] == base and r["offsets"][e + 1] == base + block
+            assert np.array_equal(st[base:base + keep.size], keep // k_max)
+            assert np.all(st[base + keep.size:base + block] == -1)
+            assert np.array_equal(dp[keep], base + np.arange(keep.size))
+            assert np.all(dp[slots[keep.size:]] == -1)
+            base += block
+        assert r["dropped"] == dropped and st.size == base
+        assert np.all(dp[flat < 0] == -1)
+        if cap <= 0 and pad == 1:  # no limit, no padding: the plain dispatch
+            q = oracle.dispatch(ids, E)
+            for key in ("counts", "offsets", "sorted_token", "dest_pos"):
+                assert np.array_equal(r[key], q[key])
+    r = oracle.dispatch_limited(np.array([[0, 5], [1, -1]], np.int32), 4, capacity=1, pad=2)
+    assert r["status"] == oracle.ERR_INDEX
+
+
+def pin_ep_layout():
+    # Worked by hand: 2 ranks, 4 experts (rank 0 owns 0-1, rank 1 owns 2-3),
+    # 3 tokens x 2 slots each.  Owner 0 receives expert 0 from rank 0 (slots
+    # 0, 5) then rank 1 (slot 2), then expert 1 from rank 0 (slot 4) and rank 1
+    # (slot 1); owner 1 receives expert 2 (rank 0 slot 2, rank 1 slot 3), then
+    # expert 3 (rank 0 slot 1, rank 1 slots 0, 4, 5).
+    ids = np.array([[[0, 3], [2, -1], [1, 0]], [[3, 1], [0, 2], [3, 3]]], np.int32)
+    r = oracle.ep_layout(ids, 4)
+    assert r["status"] == oracle.OK
+    assert r["dest_rank"].tolist() == [[[0, 1], [1, -1], [0, 0]], [[1, 0], [0, 1], [1, 1]]]
+    assert r["dest_row"].tolist() == [[[0, 2], [0, -1], [3, 1]], [[3, 4], [2, 1], [4, 5]]]
+    assert r["recv_rows"].tolist() == [5, 6]
+    # One rank: the plain dispatch.  Several: the order of a sort by
+    # (expert, source rank, flat slot) restricted to each owner.
+    rng = np.random.default_rng(47)
+    for G, T, k_max, E in ((1, 50, 3, 8), (2, 40, 2, 8), (4, 64, 4, 16), (8, 33, 6, 64)):
+        ids = rng.integers(0, E, size=(G, T, k_max)).astype(np.int32)
+        ids[rng.random(size=ids.shape) < 0.1] = -1
+        r = oracle.ep_layout(ids, E)
+        if G == 1:
+            assert np.array_equal(r["dest_row"][0], oracle.dispatch(ids[0], E)["dest_pos"])
+        el = E // G
+        src_r, src_a = np.nonzero(ids.reshape(G, -1) >= 0)
+        e = ids.reshape(G, -1)[src_r, src_a]
+        order = np.lexsort((src_a, src_r, e))
+        owner = e[order] // el
+        for d in range(G):
+            mine = order[owner == d]
+            rows = r["dest_row"].reshape(G, -1)[src_r[mine], src_a[mine]]
+            assert np.array_equal(rows, np.arange(mine.size))
+            assert np.all(r["dest_rank"].reshape(G, -1)[src_r[mine], src_a[mine]] == d)
+            assert r["recv_rows"][d] == mine.size
+        assert np.all(r["dest_rank"][ids < 0] == -1) and np.all(r["dest_row"][ids < 0] == -1)
+    # The exchange round trip: identity experts (y = received x) and weights
+    # summing to 1 give every token back exactly.
+    G, T, k_max, E, d = 4, 24, 3, 16, 16
+    ids = np.stack([np.stack([rng.permutation(E)[:k_max] for _ in range(T)]) for _ in range(G)])
+    r = oracle.ep_layout(ids.astype(np.int32), E)
+    x = _bf16_bits_from_f32(rng.normal(size=(G, T, d)).astype(np.float32))
+    recv = oracle.ep_permute(x, r["dest_rank"], r["dest_row"], r["recv_rows"])
+    w = np.full((G, T, k_max), 0.25, np.float32)
+    w[..., 0] = 0.5
+    outs = oracle.ep_combine(recv, w, r["dest_rank"], r["dest_row"], want_mag=False)
+    for g in range(G):
+        assert np.array_equal(outs[g], _bits_to_f64(x[g]))
+
+
 # ---------------------------------------------------------------- permute
 def pin_permute_copy():
     rng = np.random.default_rng(51)
@@ -430,6 +574,7 @@ def pin_combine_cases():
 
 PINS = [pin_score_closed_forms, pin_score_library_cases, pin_status_and_nan,
         pin_gate_integer_exact, pin_gate_torch_fp64, pin_hash_lookup, pin_dispatch_library,
+        pin_dispatch_limited, pin_ep_layout, pin_route_grouped,
         pin_permute_copy, pin_combine_cases, pin_weight_invariants, pin_dynamic_k_prefix,
         pin_deepseek_worked_cases, pin_brute_force_selection]
 

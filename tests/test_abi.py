@@ -90,3 +90,18 @@ def test_host_validation_needs_no_gpu(lib):
 def test_binding_fails_loudly_without_library(tmp_path):
     with pytest.raises(RuntimeError, match="missing"):
         moe.load_library(str(tmp_path / "libmoe_dispatch.so"))
+
+
+def test_limited_rows_bound(lib):
+    # min(T*k, E*capacity) + E*(pad-1)
+    assert moe.moe_dispatch_limited_rows(100, 2, 8) == 200
+    assert moe.moe_dispatch_limited_rows(100, 2, 8, capacity=10) == 80
+    assert moe.moe_dispatch_limited_rows(100, 2, 8, capacity=30, pad=128) == 200 + 8 * 127
+    assert moe.moe_dispatch_limited_rows(0, 4, 16, capacity=5, pad=4) == 16 * 3
+    for bad in (dict(capacity=-1), dict(pad=0), dict(pad=4097)):
+        with pytest.raises(moe.MoeError):
+            moe.moe_dispatch_limited_rows(10, 2, 8, **bad)
+    with pytest.raises(moe.MoeError):
+        moe.moe_dispatch_limited_rows(1 << 27, 16, 8)  # T*k_max reaches 2^31
+    assert moe.switch_capacity(262144, 1, 128, 1.0) == 2048
+    assert moe.switch_capacity(256, 2, 8, 1.25) == 80

@@ -1,0 +1,66 @@
+"""bench.py's host-side pieces without a GPU: the byte model each roofline
+fraction divides by, and the oracle chain its CPU baseline and reference arm
+time (run here on small CPU-generated samples of every workload)."""
+import importlib.util
+import os
+
+import numpy as np
+import pytest
+
+from token_dispatch_moe_b200.workloads import WORKLOADS, expert_rows, make_inputs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_stage_bytes_qwen3(bench):
+    wl = WORKLOADS["qwen3_dynk"]
+    T, d, E, k = 16384, 2048, 128, 16
+    n = 150000
+    b = bench.stage_bytes(wl, n, fused=False)
+    assert b["gate_gemm"] == T * d * 2 + E * d * 2 + T * E * 4
+    assert b["route"] == T * E * 4 + T * k * 8 + T * 4
+    assert b["permute"] == T * d * 2 + n * d * 2 + T * k * 4
+    assert b["combine"] == n * d * 2 + T * d * 2 + 8 * T * k
+    f = bench.stage_bytes(wl, n, fused=True)
+    assert "gate_gemm" not in f and "route" not in f
+    assert f["gate_route"] == T * d * 2 + E * d * 2 + T * k * 8 + T * 4
+
+
+def test_stage_bytes_capacity(bench):
+    wl = WORKLOADS["llama4_top1_capacity"]
+    T, d, E = wl.T, wl.d, wl.E
+    kept, t_read, pad_rows = 250000, 250000, 5000
+    b = bench.stage_bytes(wl, T, limited=(kept, t_read, pad_rows))
+    assert b["permute"] == t_read * d * 2 + kept * d * 2 + T * 4
+    assert b["combine"] == kept * d * 2 + T * d * 2 + T * d * 2 + 8 * T
+    assert b["dispatch"] == T * 4 + kept * 4 + T * 4 + 8 * E + pad_rows * 4
+    assert wl.capacity == T // E  # factor 1.0: the fair share
+
+
+def test_expert_rows_bound():
+    wl = WORKLOADS["llama4_top1_capacity"].scaled(1000)
+    assert wl.capacity == 8  # ceil(1000 / 128)
+    assert expert_rows(wl, None) == min(1000, 128 * 8) + 128 * 127
+    assert expert_rows(WORKLOADS["gptoss_top4"].scaled(10), None) == 40
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_oracle_chain_runs_on_cpu_inputs(bench, name):
+    wl = WORKLOADS[name].scaled(300)
+    inp = make_inputs(wl, "cpu")
+    h = bench.oracle_inputs(wl, inp, 40)
+    assert h["T"] == 40 and h["x"].shape == (40, wl.d)
+    n = int(h["kpt"].sum()) if wl.k_choices else 40 * wl.k_max
+    assert h["y"].shape[0] >= n
+    bench.oracle_chain(wl, h)
+    assert bench.oracle_sample_size(wl, inp, 0.05) >= 8
+    if wl.k_choices:
+        assert set(np.unique(h["kpt"])) <= set(wl.k_choices)

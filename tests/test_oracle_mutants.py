@@ -48,6 +48,18 @@ MUTANTS = {
                           "int32_t pos = offsets[e + 1] - 1 - seen[e];"),
     "offsets_off_by_one": ("offsets[e + 1] = offsets[e] + counts[e];",
                            "offsets[e + 1] = offsets[e] + counts[e] - (e == E - 1);"),
+    "capacity_keeps_last": ("if (capacity > 0 && rank >= capacity) continue;",
+                            "if (capacity > 0 && counts[e] - 1 - rank >= capacity) continue;"),
+    "capacity_block_unpadded": ("int32_t block = (kept + pad - 1) / pad * pad;",
+                                "int32_t block = kept / pad * pad + (kept % pad ? 1 : 0);"),
+    "capacity_demand_clipped": ("            *dropped += kept - capacity;\n            kept = capacity;",
+                                "            *dropped += kept - capacity;\n            kept = capacity;\n            counts[e] = capacity;"),
+    "grouped_candidates_worst": ("cand[nc++] = grp[i];", "cand[nc++] = grp[gsz - 1 - i];"),
+    "grouped_no_final_sort": ("        qsort(cand, (size_t)nc, sizeof(ranked), by_key_desc);\n        int32_t *sel = ids + t * k_max;",
+                              "        int32_t *sel = ids + t * k_max;"),
+    "ep_owner_modulo": ("const int32_t d = e / el;", "const int32_t d = e % G;"),
+    "ep_sources_reversed": ("if (ids_all[(int64_t)r * n + a] == e) {",
+                            "if (ids_all[(int64_t)(G - 1 - r) * n + a] == e) {"),
     "permute_wrong_row": ("memcpy(xs + (int64_t)pos * d, x + t * (int64_t)d,",
                           "memcpy(xs + (int64_t)pos * d, x + ((t + 1) % T) * (int64_t)d,"),
     "combine_drops_shared": ("acc += sv;", "acc += 0.0 * sv;"),

@@ -94,8 +94,11 @@ def test_route_parity(case):
     logits[::17] = torch.round(logits[::17] * 2) / 2  # rows with many exact ties
     logits[5] = 0.0                                   # a row where every key ties
     bias = (torch.rand((E,), generator=g, device=DEV) * 0.2 - 0.1) if has_bias else None
-    kpt = torch.randint(0, k_max + 1, (T,), generator=g, device=DEV,
-                        dtype=torch.int32) if dyn else None
+    if dyn == "seg":
+        kpt = _seg_k(T, k_max)
+    else:
+        kpt = torch.randint(0, k_max + 1, (T,), generator=g, device=DEV,
+                            dtype=torch.int32) if dyn else None
     p = moe.RouteParams.make(E, k_max, score, G, TG, topn, renorm, scale)
     ids = torch.full((T, k_max), -7, dtype=torch.int32, device=DEV)
     w = torch.full((T, k_max), 7.0, device=DEV)
@@ -245,6 +248,74 @@ def test_dispatch_edge_cases():
 
 
 # ---------------------------------------------------------- permute / combine
+@pytest.mark.parametrize("T,k,E,cap,pad,hot", [
+    (1, 1, 4, 0, 1, False), (3001, 1, 128, 0, 128, True), (70000, 1, 128, 547, 128, True),
+    (5000, 8, 64, 400, 16, False), (777, 6, 384, 3, 1, True), (40000, 4, 128, 1, 7, True),
+    (20000, 16, 512, 0, 64, False), (9000, 2, 8, 2250, 128, True)])
+def test_dispatch_limited_parity(T, k, E, cap, pad, hot):
+    """Capacity cut and block padding, bit-exact against the oracle."""
+    g = _gen(T * 7 + E + cap + pad)
+    ids = torch.randint(0, E, (T, k), generator=g, device=DEV, dtype=torch.int32)
+    if hot:  # a few experts take most of the demand, so the cut bites
+        sel = torch.rand((T, k), generator=g, device=DEV) < 0.5
+        ids = torch.where(sel, ids % 4, ids)
+    ids[torch.rand((T, k), generator=g, device=DEV) < 0.1] = -1
+    rows = moe.moe_dispatch_limited_rows(T, k, E, cap, pad)
+    counts = torch.full((E,), -7, dtype=torch.int32, device=DEV)
+    offsets = torch.full((E + 1,), -7, dtype=torch.int32, device=DEV)
+    sorted_token = torch.full((max(rows, 1),), -7, dtype=torch.int32, device=DEV)
+    dest = torch.full((T, k), -7, dtype=torch.int32, device=DEV)
+    dropped = torch.full((1,), -7, dtype=torch.int32, device=DEV)
+    ws = torch.empty((max(moe.moe_dispatch_workspace_size(T, k, E), 256),), dtype=torch.uint8,
+                     device=DEV)
+    st = _status()
+    moe.moe_dispatch_limited(ids, E, cap, pad, counts, offsets, sorted_token, dest, ws, dropped, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    o = oracle.dispatch_limited(ids.cpu().numpy(), E, capacity=cap, pad=pad)
+    n = int(o["offsets"][-1])
+    assert np.array_equal(counts.cpu().numpy(), o["counts"])
+    assert np.array_equal(offsets.cpu().numpy(), o["offsets"])
+    assert np.array_equal(sorted_token.cpu().numpy()[:n], o["sorted_token"])
+    assert np.array_equal(dest.cpu().numpy(), o["dest_pos"])
+    assert dropped.item() == o["dropped"]
+    if cap == 0 and pad == 1:
+        ref = _dispatch(ids, E)
+        assert torch.equal(dest, ref[3])
+
+
+def test_dispatch_limited_then_permute_combine():
+    """Dropped slots are skipped by permute and combine; padding rows untouched."""
+    T, k, E, d, cap, pad = 2000, 2, 16, 256, 200, 128
+    g = _gen(99)
+    ids = torch.randint(0, 4, (T, k), generator=g, device=DEV, dtype=torch.int32)
+    rows = moe.moe_dispatch_limited_rows(T, k, E, cap, pad)
+    counts = torch.empty((E,), dtype=torch.int32, device=DEV)
+    offsets = torch.empty((E + 1,), dtype=torch.int32, device=DEV)
+    sorted_token = torch.empty((rows,), dtype=torch.int32, device=DEV)
+    dest = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    ws = torch.empty((max(moe.moe_dispatch_workspace_size(T, k, E), 256),), dtype=torch.uint8,
+                     device=DEV)
+    moe.moe_dispatch_limited(ids, E, cap, pad, counts, offsets, sorted_token, dest, ws)
+    x = torch.randn((T, d), generator=g, device=DEV).to(torch.bfloat16)
+    xs = torch.full((rows, d), 3.0, dtype=torch.bfloat16, device=DEV)
+    moe.moe_permute(x, dest, xs)
+    w = torch.rand((T, k), generator=g, device=DEV)
+    out = torch.empty((T, d), dtype=torch.bfloat16, device=DEV)
+    moe.moe_combine(xs, w, dest, None, out)
+    torch.cuda.synchronize()
+    n = int(offsets[-1].item())
+    st = sorted_token[:n].cpu().numpy()
+    xs_c = xs[:n].cpu()
+    x_c = x.cpu()
+    kept = st >= 0
+    assert torch.equal(xs_c[torch.from_numpy(kept)], x_c[torch.from_numpy(st[kept]).long()])
+    assert torch.all(xs_c[torch.from_numpy(~kept)] == 3.0)
+    dropped_rows = (dest.cpu().numpy() < 0).all(axis=1)
+    assert dropped_rows.any() and np.all(out.float().cpu().numpy()[dropped_rows] == 0.0)
+    check_combine(out, xs, w.cpu().numpy(), dest.cpu().numpy())
+
+
 @pytest.mark.parametrize("T,k,d,E", [(1, 1, 8, 4), (999, 8, 2048, 64), (500, 6, 7168, 384),
                                      (1234, 4, 2880, 128), (100, 32, 136, 512),
                                      (257, 2, 128, 8)])
@@ -302,3 +373,98 @@ def test_route_keys_equal_in_high_bits(k_max, score, has_bias):
     r = check_route(ids.cpu().numpy(), w.cpu().numpy(), logits.cpu().numpy(), k_max=k_max,
                     score=score, bias=None if bias is None else bias.cpu().numpy())
     print(r)
+
+
+# ------------------------------------------------------- fused gate + route
+FUSED_CASES = [
+    # T, d, E, k_max, score, bias, G, TG, topn, renorm, scale, dyn, integer_inputs
+    (515, 2048, 128, 16, "softmax", False, 1, 1, 1, True, 1.0, True, False),
+    (300, 7168, 256, 8, "sigmoid", True, 8, 4, 2, True, 2.5, False, False),
+    (260, 7168, 384, 6, "sqrt_softplus", False, 1, 1, 1, True, 1.0, False, False),
+    (333, 512, 128, 4, "topk_softmax", False, 1, 1, 1, True, 1.0, False, False),
+    (129, 256, 128, 1, "sigmoid", False, 1, 1, 1, False, 1.0, False, False),
+    (200, 1024, 8, 2, "softmax", False, 1, 1, 1, True, 1.0, False, False),
+    (140, 512, 30, 5, "softmax", True, 3, 2, 2, True, 1.0, True, False),
+    (257, 256, 512, 16, "sigmoid", True, 32, 8, 2, True, 1.0, False, False),
+    (300, 128, 128, 8, "softmax", False, 1, 1, 1, False, 1.0, False, True),   # many exact ties
+    (300, 256, 256, 8, "sigmoid", True, 8, 4, 2, True, 2.5, True, True),      # ties + groups
+    # k fixed per 128-token block (the kernel narrows its selection per tile)
+    (900, 2048, 128, 16, "softmax", False, 1, 1, 1, True, 1.0, "seg", False),
+    (900, 512, 64, 8, "sigmoid", True, 1, 1, 1, True, 1.0, "seg", False),
+    (700, 1024, 256, 16, "sigmoid", True, 8, 4, 2, True, 2.5, "seg", True),
+]
+
+SEG_K = [4, 1, 16, 8, 3, 0, 2]
+
+
+def _seg_k(T, k_max):
+    return torch.tensor([min(SEG_K[(i // 128) % len(SEG_K)], k_max) for i in range(T)],
+                        dtype=torch.int32, device=DEV)
+
+
+@pytest.mark.parametrize("case", FUSED_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_gate_route_fused(case):
+    """moe_gate_route must pick exactly the ids moe_gate_gemm + moe_route pick,
+    with weights equal to rounding, and both must match the oracle."""
+    T, d, E, k_max, score, has_bias, G, TG, topn, renorm, scale, dyn, integer = case
+    g = _gen(T + d + E + k_max)
+    if integer:
+        x = torch.randint(-2, 3, (T, d), generator=g, device=DEV).to(torch.bfloat16)
+        w = torch.randint(-2, 3, (E, d), generator=g, device=DEV).to(torch.bfloat16)
+    else:
+        x = torch.randn((T, d), generator=g, device=DEV).to(torch.bfloat16)
+        w = (torch.randn((E, d), generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    bias = (torch.rand((E,), generator=g, device=DEV) * 0.2 - 0.1) if has_bias else None
+    if dyn == "seg":
+        kpt = _seg_k(T, k_max)
+    else:
+        kpt = torch.randint(0, k_max + 1, (T,), generator=g, device=DEV,
+                            dtype=torch.int32) if dyn else None
+    p = moe.RouteParams.make(E, k_max, score, G, TG, topn, renorm, scale)
+    ids = torch.full((T, k_max), -7, dtype=torch.int32, device=DEV)
+    wts = torch.full((T, k_max), 7.0, device=DEV)
+    logits = torch.full((T, E), float("nan"), device=DEV)
+    st = _status()
+    moe.moe_gate_route(x, w, bias, kpt, p, ids, wts, logits, st)
+    ref_logits = torch.empty((T, E), device=DEV)
+    ref_ids = torch.empty_like(ids)
+    ref_w = torch.empty_like(wts)
+    moe.moe_gate_gemm(x, w, ref_logits)
+    moe.moe_route(ref_logits, bias, kpt, p, ref_ids, ref_w)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    assert torch.equal(logits, ref_logits)
+    assert torch.equal(ids, ref_ids)
+    assert torch.allclose(wts, ref_w, rtol=2e-6, atol=0)
+    check_route(ids.cpu().numpy(), wts.cpu().numpy(), logits.cpu().numpy(), k_max=k_max,
+                score=score, bias=None if bias is None else bias.cpu().numpy(),
+                kpt=None if kpt is None else kpt.cpu().numpy(), n_groups=G, topk_groups=TG,
+                group_topn=topn, renormalize=renorm, route_scale=scale)
+
+
+def test_gate_route_without_logits_and_nan():
+    T, d, E, k = 150, 256, 64, 4
+    g = _gen(4242)
+    x = torch.randn((T, d), generator=g, device=DEV).to(torch.bfloat16)
+    x[7, 3] = float("inf")  # row 7's logits become +-inf ...
+    w = (torch.randn((E, d), generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    w[5, 3] = 0.0           # ... and inf * 0 = NaN for expert 5
+    p = moe.RouteParams.make(E, k, "sigmoid", renormalize=False)
+    ids = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    wts = torch.empty((T, k), device=DEV)
+    st = _status()
+    moe.moe_gate_route(x, w, None, None, p, ids, wts, None, st)  # logits not written
+    logits = torch.empty((T, E), device=DEV)
+    ref_ids = torch.empty_like(ids)
+    ref_w = torch.empty_like(wts)
+    moe.moe_gate_gemm(x, w, logits)
+    moe.moe_route(logits, None, None, p, ref_ids, ref_w)
+    torch.cuda.synchronize()
+    assert st.item() == moe.MOE_ERR_NAN_LOGIT
+    assert torch.equal(ids, ref_ids)
+    ok = torch.isfinite(ref_w)
+    assert torch.allclose(wts[ok], ref_w[ok], rtol=2e-6, atol=0)
+    with pytest.raises(moe.MoeError):  # k_max above the fused limit
+        moe.moe_gate_route(x, w, None, None, moe.RouteParams.make(E, 17, "softmax"),
+                           torch.empty((T, 17), dtype=torch.int32, device=DEV),
+                           torch.empty((T, 17), device=DEV))

@@ -11,15 +11,16 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_check import (check_combine, check_dispatch, check_gate, check_permute, check_route,
-                       np32)
+from gpu_check import (check_combine, check_dispatch, check_dispatch_limited, check_gate,
+                       check_permute, check_route, np32)
 from token_dispatch_moe_b200.path import RouterDispatch
 from token_dispatch_moe_b200.workloads import WORKLOADS, make_inputs
 
 pytestmark = pytest.mark.gpu
 
 REDUCED_T = {"mixtral_tiny": 253, "qwen3_dynk": 1500, "deepseek_v3": 777,
-             "deepseek_v4": 777, "llama4_top1": 3001, "gptoss_top4": 3001}
+             "deepseek_v4": 777, "llama4_top1": 3001, "gptoss_top4": 3001,
+             "llama4_top1_capacity": 3001}
 
 
 def _sample(T, n, seed):
@@ -28,9 +29,9 @@ def _sample(T, n, seed):
     return np.unique(np.concatenate([pick, [0, T - 1]]))
 
 
-def _run_and_check(wl, sampled: bool):
+def _run_and_check(wl, sampled: bool, fused=None):
     inp = make_inputs(wl, "cuda")
-    path = RouterDispatch(wl)
+    path = RouterDispatch(wl, fused=fused, keep_logits=True)
     path.run(inp)
     torch.cuda.synchronize()
     assert path.status.item() == 0, path.status.item()
@@ -46,12 +47,18 @@ def _run_and_check(wl, sampled: bool):
                                   group_topn=wl.group_topn, renormalize=wl.renormalize,
                                   route_scale=wl.route_scale)
     dest = np32(path.dest_pos)
-    n = check_dispatch(ids, np32(path.counts), np32(path.offsets), np32(path.sorted_token), dest,
-                       wl.E)
+    if wl.limited:
+        n = check_dispatch_limited(ids, np32(path.counts), np32(path.offsets),
+                                   np32(path.sorted_token), dest, path.dropped.item(), wl.E,
+                                   path.capacity, wl.pad)
+        report["dropped"] = path.dropped.item()
+    else:
+        n = check_dispatch(ids, np32(path.counts), np32(path.offsets), np32(path.sorted_token),
+                           dest, wl.E)
     tokens = _sample(wl.T, 1024, 2) if sampled else None
     check_permute(path.xs, inp["x"], dest, tokens)
     if wl.combine:
-        assert inp["y"].shape[0] == n
+        assert inp["y"].shape[0] >= n
         tokens = _sample(wl.T, 512, 3) if sampled else None
         report["combine_worst"] = check_combine(path.out, inp["y"], w, dest, inp["shared"], tokens)
     if wl.hash_vocab:
@@ -74,9 +81,12 @@ def _run_and_check(wl, sampled: bool):
     return report
 
 
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "separate"])
 @pytest.mark.parametrize("name", list(WORKLOADS))
-def test_workload_reduced(name):
-    _run_and_check(WORKLOADS[name].scaled(REDUCED_T[name]), sampled=False)
+def test_workload_reduced(name, fused):
+    if not fused and not WORKLOADS[name].gate:
+        pytest.skip("no gate: the fused and separate paths are the same")
+    _run_and_check(WORKLOADS[name].scaled(REDUCED_T[name]), sampled=False, fused=fused)
 
 
 @pytest.mark.parametrize("name", list(WORKLOADS))

@@ -12,6 +12,7 @@ call raises, telling how to build it.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 
 import torch
@@ -21,7 +22,7 @@ __all__ = [
     "SCORE_SOFTMAX", "SCORE_SIGMOID", "SCORE_SQRT_SOFTPLUS", "SCORE_TOPK_SOFTMAX",
     "MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED", "MOE_ERR_CUDA",
     "MOE_ERR_DEVICE_INDEX", "MOE_ERR_TIMEOUT", "MOE_ERR_NAN_LOGIT",
-    "moe_status_string", "moe_gate_gemm", "moe_route", "moe_hash_route",
+    "moe_status_string", "moe_gate_gemm", "moe_gate_route", "moe_route", "moe_hash_route",
     "moe_dispatch_workspace_size", "moe_dispatch", "moe_dispatch_static", "moe_permute",
     "moe_combine",
 ]
@@ -80,11 +81,18 @@ def load_library(path: str | None = None):
     sig = {
         "moe_status_string": ([st], ctypes.c_char_p),
         "moe_gate_gemm": ([P, P, P, i64, i32, i32, P, P], st),
+        "moe_gate_route": ([P, P, P, P, ctypes.POINTER(RouteParams), i64, i32, P, P, P, P, P], st),
         "moe_route": ([P, P, P, ctypes.POINTER(RouteParams), i64, P, P, P, P], st),
         "moe_hash_route": ([P, P, i32, i32, P, ctypes.POINTER(RouteParams), i64, P, P, P, P], st),
         "moe_dispatch_workspace_size": ([i64, i32, i32, ctypes.POINTER(ctypes.c_size_t)], st),
         "moe_dispatch": ([P, i64, i32, i32, P, P, P, P, P, ctypes.c_size_t, P, P], st),
         "moe_dispatch_static": ([P, i64, i32, i32, P, P, P, P, P, P], st),
+        "moe_ep_layout": ([P, P, P, P, i32, i32, i64, i32, i32, P, P, P, P, P], st),
+        "moe_ep_permute": ([P, P, P, P, i32, i64, i64, i32, i32, P, P], st),
+        "moe_ep_combine": ([P, P, P, P, P, i32, i64, i64, i32, i32, P, P, P], st),
+        "moe_dispatch_limited_rows": ([i64, i32, i32, i32, i32, ctypes.POINTER(i64)], st),
+        "moe_dispatch_limited": ([P, i64, i32, i32, i32, i32, P, P, P, i64, P, P, P,
+                                  ctypes.c_size_t, P, P], st),
         "moe_permute": ([P, P, i64, i32, i32, P, P], st),
         "moe_combine": ([P, P, P, P, i64, i32, i32, P, P], st),
     }
@@ -143,6 +151,30 @@ def moe_gate_gemm(x, w, logits, d_status=None, stream=None):
         raise ValueError("shape mismatch")
     _check(load_library().moe_gate_gemm(_ptr(x), _ptr(w), _ptr(logits), T, d, E,
                                         _ptr(d_status), _stream(stream)), "moe_gate_gemm")
+
+
+def moe_gate_route(x, w, bias, k_per_token, params: RouteParams, topk_ids, topk_w, logits=None,
+                   d_status=None, stream=None):
+    """moe_gate_gemm + moe_route in one kernel: each token's logits row is routed
+    from the tensor-core accumulator; logits are written only if given."""
+    _need(x, torch.bfloat16, "x", 2)
+    _need(w, torch.bfloat16, "w", 2)
+    _need(bias, torch.float32, "bias", 1)
+    _need(k_per_token, torch.int32, "k_per_token", 1)
+    _need(topk_ids, torch.int32, "topk_ids", 2)
+    _need(topk_w, torch.float32, "topk_w", 2)
+    _need(logits, torch.float32, "logits", 2)
+    _need(d_status, torch.int32, "d_status")
+    T, d = x.shape
+    E = w.shape[0]
+    if w.shape[1] != d or E != params.num_experts or \
+            tuple(topk_ids.shape) != (T, params.k_max) or tuple(topk_w.shape) != (T, params.k_max) \
+            or (logits is not None and tuple(logits.shape) != (T, E)):
+        raise ValueError("shape mismatch")
+    _check(load_library().moe_gate_route(_ptr(x), _ptr(w), _ptr(bias), _ptr(k_per_token),
+                                         ctypes.byref(params), T, d, _ptr(topk_ids), _ptr(topk_w),
+                                         _ptr(logits), _ptr(d_status), _stream(stream)),
+           "moe_gate_route")
 
 
 def moe_route(logits, bias, k_per_token, params: RouteParams, topk_ids, topk_w, d_status=None,
@@ -204,6 +236,98 @@ def moe_dispatch(topk_ids, E, counts, offsets, sorted_token, dest_pos, workspace
                                        _ptr(sorted_token), _ptr(dest_pos), _ptr(workspace),
                                        workspace.numel(), _ptr(d_status), _stream(stream)),
            "moe_dispatch")
+
+
+def moe_dispatch_limited_rows(T: int, k_max: int, E: int, capacity: int = 0, pad: int = 1) -> int:
+    """Rows sorted_token and the permuted activations need under moe_dispatch_limited."""
+    out = ctypes.c_int64(0)
+    _check(load_library().moe_dispatch_limited_rows(T, k_max, E, capacity, pad, ctypes.byref(out)),
+           "moe_dispatch_limited_rows")
+    return out.value
+
+
+def switch_capacity(T: int, k: int, E: int, capacity_factor: float) -> int:
+    """Per-expert capacity ceil(capacity_factor * T * k / E): the fair share of
+    the T*k slots times the factor (the Switch-style limit)."""
+    return max(1, math.ceil(capacity_factor * T * k / E))
+
+
+def moe_dispatch_limited(topk_ids, E, capacity, pad, counts, offsets, sorted_token, dest_pos,
+                         workspace, dropped=None, d_status=None, stream=None):
+    """moe_dispatch with a per-expert capacity (0 = none; each expert keeps its
+    first `capacity` slots in flat order) and expert blocks padded to a multiple
+    of `pad` rows (padding rows of sorted_token are -1)."""
+    _need(topk_ids, torch.int32, "topk_ids", 2)
+    for t, n in ((counts, "counts"), (offsets, "offsets"), (sorted_token, "sorted_token"),
+                 (dest_pos, "dest_pos"), (dropped, "dropped"), (d_status, "d_status")):
+        _need(t, torch.int32, n)
+    _need(workspace, torch.uint8, "workspace")
+    T, k_max = topk_ids.shape
+    if counts.numel() < E or offsets.numel() < E + 1 or tuple(dest_pos.shape) != (T, k_max):
+        raise ValueError("shape mismatch")
+    _check(load_library().moe_dispatch_limited(
+        _ptr(topk_ids), T, k_max, E, capacity, pad, _ptr(counts), _ptr(offsets),
+        _ptr(sorted_token), sorted_token.numel(), _ptr(dest_pos), _ptr(dropped), _ptr(workspace),
+        workspace.numel(), _ptr(d_status), _stream(stream)), "moe_dispatch_limited")
+
+
+def moe_ep_layout(all_counts, topk_ids, dest_pos, offsets, rank, dest_rank, dest_row,
+                  recv_offsets, d_status=None, stream=None):
+    """Owner rank and receive row of every slot (expert e on rank e // (E // G))."""
+    _need(all_counts, torch.int32, "all_counts", 2)
+    for t, n in ((topk_ids, "topk_ids"), (dest_pos, "dest_pos"), (offsets, "offsets"),
+                 (dest_rank, "dest_rank"), (dest_row, "dest_row"),
+                 (recv_offsets, "recv_offsets"), (d_status, "d_status")):
+        _need(t, torch.int32, n)
+    G, E = all_counts.shape
+    T, k_max = topk_ids.shape
+    if tuple(dest_pos.shape) != (T, k_max) or tuple(dest_rank.shape) != (T, k_max) or \
+            tuple(dest_row.shape) != (T, k_max) or offsets.numel() < E + 1 or \
+            recv_offsets.numel() < E // G + 1:
+        raise ValueError("shape mismatch")
+    _check(load_library().moe_ep_layout(
+        _ptr(all_counts), _ptr(topk_ids), _ptr(dest_pos), _ptr(offsets), G, rank, T, k_max, E,
+        _ptr(dest_rank), _ptr(dest_row), _ptr(recv_offsets), _ptr(d_status), _stream(stream)),
+        "moe_ep_layout")
+
+
+def peer_table(buffers, device=None) -> torch.Tensor:
+    """Device array of the G receive-buffer addresses (int64), as the EP calls
+    take it; entry r must be rank r's buffer as mapped in this process."""
+    addrs = [b.data_ptr() for b in buffers]
+    dev = device if device is not None else buffers[0].device
+    return torch.tensor(addrs, dtype=torch.int64, device=dev)
+
+
+def moe_ep_permute(x, dest_rank, dest_row, peers, recv_capacity, d_status=None, stream=None):
+    """Store every row of x into its owners' receive buffers (peers: a
+    peer_table of G [recv_capacity, d] bf16 buffers)."""
+    _need(x, torch.bfloat16, "x", 2)
+    for t, n in ((dest_rank, "dest_rank"), (dest_row, "dest_row"), (d_status, "d_status")):
+        _need(t, torch.int32, n)
+    _need(peers, torch.int64, "peers", 1)
+    T, d = x.shape
+    k_max = dest_rank.shape[1]
+    _check(load_library().moe_ep_permute(_ptr(x), _ptr(dest_rank), _ptr(dest_row), _ptr(peers),
+                                         peers.numel(), recv_capacity, T, k_max, d,
+                                         _ptr(d_status), _stream(stream)), "moe_ep_permute")
+
+
+def moe_ep_combine(peers_y, dest_rank, dest_row, topk_w, shared, out, recv_capacity,
+                   d_status=None, stream=None):
+    """moe_combine reading each slot's expert output from its owner."""
+    for t, n in ((dest_rank, "dest_rank"), (dest_row, "dest_row"), (d_status, "d_status")):
+        _need(t, torch.int32, n)
+    _need(peers_y, torch.int64, "peers_y", 1)
+    _need(topk_w, torch.float32, "topk_w", 2)
+    _need(shared, torch.bfloat16, "shared", 2)
+    _need(out, torch.bfloat16, "out", 2)
+    T, d = out.shape
+    k_max = dest_rank.shape[1]
+    _check(load_library().moe_ep_combine(_ptr(peers_y), _ptr(dest_rank), _ptr(dest_row),
+                                         _ptr(topk_w), _ptr(shared), peers_y.numel(),
+                                         recv_capacity, T, k_max, d, _ptr(out), _ptr(d_status),
+                                         _stream(stream)), "moe_ep_combine")
 
 
 def moe_dispatch_static(topk_ids, E, counts, offsets, sorted_token, dest_pos, d_status=None,

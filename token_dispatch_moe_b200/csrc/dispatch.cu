@@ -33,6 +33,7 @@ constexpr int kDispWarps = 8;
 constexpr int kMaxE = 512;
 constexpr int kBatch = 4;  // slot loads issued together per lane (items is a multiple)
 constexpr int kSumUnroll = 16;  // independent segment-total loads in flight per thread
+constexpr int kMaxPad = 4096;   // largest block padding of moe_dispatch_limited
 
 int warp_items(int64_t n_flat) {
     int items = 4;
@@ -91,16 +92,27 @@ __global__ void __launch_bounds__(kDispWarps * 32)
     }
 }
 
+// A per-expert capacity and block padding (moe_dispatch_limited); the plain
+// dispatch is cap = INT32_MAX, pad = 1 with LIMITED = false.
+struct Limits {
+    int32_t cap;       // slots kept per expert, in flat order
+    int32_t pad;       // expert blocks rounded up to a multiple of this many rows
+    int32_t *dropped;  // nullable: number of slots over capacity
+};
+
+template <bool LIMITED>
 __global__ void __launch_bounds__(kDispWarps * 32)
     dispatch_scatter_kernel(const int32_t *__restrict__ ids, int64_t n_flat, int k_max, int E,
                             int items, int64_t S, const int32_t *__restrict__ seg_total,
                             const int32_t *__restrict__ warp_hist, int32_t *__restrict__ counts,
                             int32_t *__restrict__ offsets, int32_t *__restrict__ sorted_token,
-                            int32_t *__restrict__ dest_pos) {
+                            int32_t *__restrict__ dest_pos, Limits lim) {
     __shared__ int32_t total[kMaxE + 1];
     __shared__ int32_t before[kMaxE];
     __shared__ int32_t run[kDispWarps][kMaxE];
     __shared__ int32_t wsum[kDispWarps];
+    __shared__ int32_t kept_s[LIMITED ? kMaxE : 1];
+    __shared__ int32_t drop_s;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t s = blockIdx.x;
 
@@ -136,11 +148,25 @@ __global__ void __launch_bounds__(kDispWarps * 32)
     }
     __syncthreads();
 
-    // Exclusive scan of the totals into offsets: thread i owns experts 2i, 2i+1.
+    // Exclusive scan of the block sizes (the totals, or with limits the kept
+    // slots rounded up to the padding) into offsets: thread i owns experts 2i,
+    // 2i+1.
     {
         const int i0 = 2 * threadIdx.x, i1 = i0 + 1;
-        const int32_t c0 = i0 < E ? total[i0] : 0;
-        const int32_t c1 = i1 < E ? total[i1] : 0;
+        const int32_t n0 = i0 < E ? total[i0] : 0;
+        const int32_t n1 = i1 < E ? total[i1] : 0;
+        int32_t c0 = n0, c1 = n1;
+        if (LIMITED) {
+            if (threadIdx.x == 0) drop_s = 0;
+            const int32_t k0 = min(n0, lim.cap), k1 = min(n1, lim.cap);
+            if (i0 < E) kept_s[i0] = k0;
+            if (i1 < E) kept_s[i1] = k1;
+            c0 = (k0 + lim.pad - 1) / lim.pad * lim.pad;
+            c1 = (k1 + lim.pad - 1) / lim.pad * lim.pad;
+            __syncthreads();
+            const int32_t over = (n0 - k0) + (n1 - k1);
+            if (blockIdx.x == 0 && over) atomicAdd(&drop_s, over);
+        }
         const int32_t v = c0 + c1;
         int32_t incl = v;
 #pragma unroll
@@ -155,17 +181,18 @@ __global__ void __launch_bounds__(kDispWarps * 32)
         const int32_t excl = pre + incl - v;
         if (blockIdx.x == 0) {
             if (i0 < E) {
-                counts[i0] = c0;
+                counts[i0] = n0;
                 offsets[i0] = excl;
             }
             if (i1 < E) {
-                counts[i1] = c1;
+                counts[i1] = n1;
                 offsets[i1] = excl + c0;
             }
             if (threadIdx.x == 0) {
                 int32_t all = 0;
                 for (int w = 0; w < kDispWarps; ++w) all += wsum[w];
                 offsets[E] = all;
+                if (LIMITED && lim.dropped) *lim.dropped = drop_s;
             }
         }
         // Each warp's starting position per expert: offset + earlier segments +
@@ -175,13 +202,24 @@ __global__ void __launch_bounds__(kDispWarps * 32)
         if (i1 < E) total[i1] = excl + c0;
         __syncthreads();
     }
+    if (LIMITED) {
+        // The padding rows of expert blocks (experts shared out over blocks).
+        for (int e = (int)blockIdx.x; e < E; e += (int)gridDim.x) {
+            const int32_t lo = total[e] + kept_s[e];
+            const int32_t hi = total[e] + (kept_s[e] + lim.pad - 1) / lim.pad * lim.pad;
+            for (int32_t p = lo + (int32_t)threadIdx.x; p < hi; p += (int32_t)blockDim.x)
+                sorted_token[p] = -1;
+        }
+    }
+    // Each warp's first rank per expert (earlier segments + earlier warps of
+    // this segment); without limits the block offset is folded in as well.
     const int32_t *wh = warp_hist + s * kDispWarps * E;
     int32_t *r = run[warp];
     for (int e = lane; e < E; e += 32) {
         int32_t v[kDispWarps];
 #pragma unroll
         for (int w = 0; w < kDispWarps; ++w) v[w] = w < warp ? wh[w * E + e] : 0;
-        int32_t b = total[e] + before[e];
+        int32_t b = (LIMITED ? 0 : total[e]) + before[e];
 #pragma unroll
         for (int w = 0; w < kDispWarps; ++w) b += v[w];
         r[e] = b;
@@ -202,8 +240,9 @@ __global__ void __launch_bounds__(kDispWarps * 32)
             const int e = eb[j];
             const unsigned peers = __match_any_sync(MOE_FULL_MASK, e);
             if (e >= 0) {
-                const int32_t pos = r[e] + __popc(peers & lower);
-                sorted_token[pos] = (int32_t)(a / k_max);
+                int32_t pos = r[e] + __popc(peers & lower);
+                if (LIMITED) pos = pos < lim.cap ? total[e] + pos : -1;
+                if (pos >= 0) sorted_token[pos] = (int32_t)(a / k_max);
                 dest_pos[a] = pos;
             } else if (a < n_flat) {
                 dest_pos[a] = -1;
@@ -254,13 +293,74 @@ extern "C" moe_status moe_dispatch(const int32_t *topk_ids, int64_t T, int32_t k
         dispatch_count_kernel<<<(unsigned)S, kDispWarps * 32, 0, cs>>>(topk_ids, n_flat, E, items,
                                                                       seg_total, warp_hist,
                                                                       d_status);
-        dispatch_scatter_kernel<<<(unsigned)S, kDispWarps * 32, 0, cs>>>(
+        dispatch_scatter_kernel<false><<<(unsigned)S, kDispWarps * 32, 0, cs>>>(
             topk_ids, n_flat, k_max, E, items, S, seg_total, warp_hist, counts, offsets,
-            sorted_token, dest_pos);
+            sorted_token, dest_pos, Limits{INT32_MAX, 1, nullptr});
     } else {
         // No slots: every count and every offset is 0.
         if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, cs) != cudaSuccess ||
             cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), cs) != cudaSuccess) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
+    }
+    return launch_status();
+}
+
+// ------------------------------------------- dispatch with capacity/padding
+extern "C" moe_status moe_dispatch_limited_rows(int64_t T, int32_t k_max, int32_t E,
+                                                int32_t capacity, int32_t pad, int64_t *rows) {
+    using namespace moe;
+    if (!rows || T < 0 || k_max < 0 || k_max > 32 || E < 1 || E > kMaxE || capacity < 0 ||
+        pad < 1 || pad > kMaxPad)
+        return MOE_ERR_INVALID_ARG;
+    const int64_t n_flat = T * (int64_t)k_max;
+    int64_t kept = n_flat;
+    if (capacity > 0 && (int64_t)capacity * E < kept) kept = (int64_t)capacity * E;
+    const int64_t r = kept + (int64_t)E * (pad - 1);
+    if (n_flat >= (int64_t)INT32_MAX || r >= (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+    *rows = r;
+    return MOE_OK;
+}
+
+extern "C" moe_status moe_dispatch_limited(const int32_t *topk_ids, int64_t T, int32_t k_max,
+                                           int32_t E, int32_t capacity, int32_t pad,
+                                           int32_t *counts, int32_t *offsets,
+                                           int32_t *sorted_token, int64_t sorted_rows,
+                                           int32_t *dest_pos, int32_t *dropped, void *workspace,
+                                           size_t ws_bytes, int32_t *d_status,
+                                           moe_stream_t stream) {
+    using namespace moe;
+    int64_t bound = 0;
+    moe_status st = moe_dispatch_limited_rows(T, k_max, E, capacity, pad, &bound);
+    if (st != MOE_OK) return st;
+    size_t need = 0;
+    st = moe_dispatch_workspace_size(T, k_max, E, &need);
+    if (st != MOE_OK) return st;
+    if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
+    const int64_t n_flat = T * (int64_t)k_max;
+    if (n_flat > 0 && (!topk_ids || !sorted_token || !dest_pos || !workspace))
+        return MOE_ERR_INVALID_ARG;
+    if (n_flat > 0 && ((reinterpret_cast<uintptr_t>(workspace) & 255u) || ws_bytes < need ||
+                       sorted_rows < bound))
+        return MOE_ERR_INVALID_ARG;
+    cudaStream_t cs = as_cuda(stream);
+    const int items = warp_items(n_flat);
+    const int64_t S = num_segments(n_flat, items);
+    if (S > 0) {
+        int32_t *seg_total = static_cast<int32_t *>(workspace);
+        int32_t *warp_hist = seg_total + S * E;
+        dispatch_count_kernel<<<(unsigned)S, kDispWarps * 32, 0, cs>>>(topk_ids, n_flat, E, items,
+                                                                      seg_total, warp_hist,
+                                                                      d_status);
+        const Limits lim{capacity > 0 ? capacity : INT32_MAX, pad, dropped};
+        dispatch_scatter_kernel<true><<<(unsigned)S, kDispWarps * 32, 0, cs>>>(
+            topk_ids, n_flat, k_max, E, items, S, seg_total, warp_hist, counts, offsets,
+            sorted_token, dest_pos, lim);
+    } else {
+        if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, cs) != cudaSuccess ||
+            cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), cs) != cudaSuccess ||
+            (dropped && cudaMemsetAsync(dropped, 0, sizeof(int32_t), cs) != cudaSuccess)) {
             cudaGetLastError();
             return MOE_ERR_CUDA;
         }

@@ -140,6 +140,31 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Loads without the wait, so two loads can be in flight before one wait.
+__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -147,21 +172,375 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+// ------------------------------------------------------- fused route epilogue --
+// moe_gate_route: the route of moe_route computed in the GEMM epilogue.  A
+// TMEM lane holds one token's whole logits row, so each epilogue thread routes
+// its own row without any warp-wide step:
+//   pass 1  (optional) logits out, NaN flag, row max; softmax denominator when
+//           a key or a weight needs it; group scores (top-2 or amax of each
+//           contiguous group, in expert order) and the kept groups;
+//   pass 2  the P largest keys of kept experts with a branch-free max/min
+//           network on fp32 values (fmaxf/fminf are exact), which gives the
+//           exact k_t-th largest key tau and how many keys exceed it;
+//   pass 3  in expert-id order, every key > tau and the first (k_t - #(> tau))
+//           keys == tau (equal keys -> lower id) are appended to a per-thread
+//           list in shared memory;
+//   then the k_t entries are sorted by (key desc, id asc) and weighted.
+// Keys are recomputed from the logits in each pass (for the monotone case the
+// key is the logit itself).  NaN keys rank below every number: they enter only
+// if fewer than k_t other experts remain.
+struct FusedArgs {
+    const float *bias;
+    const int32_t *kpt;
+    int32_t *ids;
+    float *w;
+    float *logits;  // optional copy of the logits
+    int k_max, score, G, TG, topn, renorm, keys_from_scores, gsz;
+    float scale;
+};
+
+struct RowStats {
+    float m, z;  // row max and softmax denominator (when needed)
+};
+
+template <bool MONO>
+__device__ __forceinline__ float fused_key(const FusedArgs &f, float l, int e, const RowStats &st,
+                                           float zinv) {
+    if (MONO) return l;
+    float x;
+    if (f.score == MOE_SCORE_SOFTMAX)
+        x = expf(l - st.m) * zinv;
+    else if (f.score == MOE_SCORE_SIGMOID)
+        x = __frcp_rn(1.0f + expf(-l));
+    else if (f.score == MOE_SCORE_SQRT_SOFTPLUS)
+        x = sqrt_softplus_score(l);
+    else
+        x = l;
+    return x + (f.bias ? __ldg(f.bias + e) : 0.0f);
+}
+
+__device__ __forceinline__ uint32_t fkey_bits(float v) {
+    uint32_t u = __float_as_uint(v);
+    u = (v == 0.0f) ? 0u : u;
+    const uint32_t o = u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);
+    return (v != v) ? 1u : o;
+}
+
+// Bit i set when expert c0 + i exists and its group is kept.
+template <bool GROUPED>
+__device__ __forceinline__ uint32_t chunk_mask(uint32_t kept, int c0, int E, int gsz) {
+    const uint32_t valid = E - c0 >= 16 ? 0xffffu : (E > c0 ? (1u << (E - c0)) - 1u : 0u);
+    if (!GROUPED) return valid;
+    uint32_t m = 0u;
+    int g = c0 / gsz;
+    for (int start = g * gsz; start < c0 + 16 && start < E; ++g, start += gsz) {
+        if ((kept >> g) & 1u) {
+            const int lo = start > c0 ? start - c0 : 0;
+            const int hi = start + gsz < c0 + 16 ? start + gsz - c0 : 16;
+            m |= ((hi >= 32 ? 0xffffffffu : (1u << hi) - 1u)) & ~((1u << lo) - 1u);
+        }
+    }
+    return m & valid;
+}
+
+// Loads 16 columns of values (keys when keys sit in TMEM, else logits) and
+// converts them to keys.
+template <bool MONO>
+__device__ __forceinline__ void chunk_keys(const FusedArgs &f, uint32_t trow, uint32_t koff,
+                                           bool keys_in_tmem, int c0, int E, const RowStats &st,
+                                           float zinv, float (&x)[16], float (&l)[16],
+                                           bool need_logits) {
+    uint32_t r[16], q[16];
+    if (MONO || !keys_in_tmem) {
+        tmem_ld16_nowait(trow + (uint32_t)c0, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            l[i] = __uint_as_float(r[i]);
+            x[i] = (c0 + i < E) ? fused_key<MONO>(f, l[i], c0 + i, st, zinv) : -INFINITY;
+        }
+    } else {
+        tmem_ld16_nowait(trow + koff + (uint32_t)c0, q);
+        if (need_logits) tmem_ld16_nowait(trow + (uint32_t)c0, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            x[i] = __uint_as_float(q[i]);
+            l[i] = need_logits ? __uint_as_float(r[i]) : 0.0f;
+        }
+    }
+}
+
+template <int P, bool MONO, bool GROUPED>
+__device__ __forceinline__ void route_epilogue(const GemmArgs &g, const FusedArgs &f,
+                                               uint32_t trow, int64_t row, bool valid, int tid,
+                                               float *gs_s, float *lk, int32_t *li, float *ll) {
+    const int E = g.E;
+    const int ncols = g.NC * g.BN;
+    const uint32_t koff = (uint32_t)ncols;  // key columns follow the logits when stored
+    const bool keys_in_tmem = !MONO && 2 * ncols <= g.tmem_cols;
+    int kt = f.k_max;
+    if (valid && f.kpt) {
+        kt = f.kpt[row];
+        if (kt < 0 || kt > f.k_max) {
+            report(g.status, MOE_ERR_DEVICE_INDEX);
+            kt = kt < 0 ? 0 : f.k_max;
+        }
+    }
+    if (!valid) kt = 0;
+
+    // Pass 1: logits out, NaN, row max.
+    bool nan = false;
+    RowStats st{-INFINITY, 1.0f};
+    const bool vec = (E & 3) == 0;
+    for (int c0 = 0; c0 < ncols; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16_nowait(trow + (uint32_t)c0, r);
+        tmem_wait_ld();
+        if (valid && f.logits) {
+            float *dst = f.logits + row * E + c0;
+            if (vec && c0 + 16 <= E) {
+#pragma unroll
+                for (int i = 0; i < 16; i += 4)
+                    *reinterpret_cast<float4 *>(dst + i) =
+                        make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
+                                    __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    if (c0 + i < E) dst[i] = __uint_as_float(r[i]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if (c0 + i < E) {
+                const float v = __uint_as_float(r[i]);
+                nan |= v != v;
+                st.m = fmaxf(st.m, v);
+            }
+    }
+    if (valid && nan) report(g.status, MOE_ERR_NAN_LOGIT);
+    if (f.score == MOE_SCORE_SOFTMAX && (!MONO || !f.renorm)) {
+        float z = 0.0f;
+        for (int c0 = 0; c0 < ncols; c0 += 16) {
+            uint32_t r[16];
+            tmem_ld16_nowait(trow + (uint32_t)c0, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (c0 + i < E) z += expf(__uint_as_float(r[i]) - st.m);
+        }
+        st.z = z;
+    }
+    const float zinv = 1.0f / st.z;
+
+    // Keys into spare TMEM columns (score keys only), group scores, kept groups.
+    if (!MONO && keys_in_tmem) {
+        for (int c0 = 0; c0 < ncols; c0 += 16) {
+            uint32_t r[16];
+            tmem_ld16_nowait(trow + (uint32_t)c0, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                r[i] = __float_as_uint(fused_key<MONO>(f, __uint_as_float(r[i]), c0 + i, st, zinv));
+            tmem_st16(trow + koff + (uint32_t)c0, r);
+        }
+        tmem_wait_st();
+    }
+    uint32_t kept = 0xffffffffu;
+    if (GROUPED) {
+        float t1 = -INFINITY, t2 = -INFINITY;
+        int gpos = 0, gidx = 0;  // position within the current group, group index
+        for (int c0 = 0; c0 < ncols; c0 += 16) {
+            float x[16], l[16];
+            chunk_keys<MONO>(f, trow, koff, keys_in_tmem, c0, E, st, zinv, x, l, false);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                if (c0 + i < E) {
+                    if (x[i] > t1) {
+                        t2 = t1;
+                        t1 = x[i];
+                    } else if (x[i] > t2) {
+                        t2 = x[i];
+                    }
+                    if (++gpos == f.gsz) {
+                        gs_s[gidx * 128 + tid] = f.topn == 1 ? t1 : t1 + t2;
+                        t1 = t2 = -INFINITY;
+                        gpos = 0;
+                        ++gidx;
+                    }
+                }
+            }
+        }
+        kept = 0u;
+        for (int r = 0; r < f.TG; ++r) {
+            uint32_t bk = 0u;
+            int bg = 0;
+            for (int gg = 0; gg < f.G; ++gg) {
+                const uint32_t k = ((kept >> gg) & 1u) ? 0u : fkey_bits(gs_s[gg * 128 + tid]);
+                if (k > bk) {
+                    bk = k;
+                    bg = gg;
+                }
+            }
+            kept |= 1u << bg;
+        }
+    }
+
+    // Pass 2: the P largest keys (values only; NaN counts as -inf here).
+    float L[P];
+#pragma unroll
+    for (int p = 0; p < P; ++p) L[p] = -INFINITY;
+    for (int c0 = 0; c0 < ncols; c0 += 16) {
+        float x[16], l[16];
+        chunk_keys<MONO>(f, trow, koff, keys_in_tmem, c0, E, st, zinv, x, l, false);
+        const uint32_t cm = chunk_mask<GROUPED>(kept, c0, E, f.gsz);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float v = ((cm >> i) & 1u) ? x[i] : -INFINITY;
+            v = (v != v) ? -INFINITY : v;
+#pragma unroll
+            for (int p = 0; p < P; ++p) {
+                const float hi = fmaxf(L[p], v);
+                v = fminf(L[p], v);
+                L[p] = hi;
+            }
+        }
+    }
+    float tau = -INFINITY;
+    int n_gt = 0;
+#pragma unroll
+    for (int p = 0; p < P; ++p)
+        if (p == kt - 1) tau = L[p];
+#pragma unroll
+    for (int p = 0; p < P; ++p) n_gt += (p < kt && L[p] > tau) ? 1 : 0;
+    const int need_eq = kt - n_gt;
+
+    // Pass 3: collect the selected experts in id order.
+    int cnt = 0, eq_seen = 0;
+    if (__any_sync(MOE_FULL_MASK, kt > 0)) {
+        for (int c0 = 0; c0 < ncols; c0 += 16) {
+            float x[16], l[16];
+            chunk_keys<MONO>(f, trow, koff, keys_in_tmem, c0, E, st, zinv, x, l, true);
+            const uint32_t cm = kt > 0 ? chunk_mask<GROUPED>(kept, c0, E, f.gsz) : 0u;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                if ((cm >> i) & 1u) {
+                    const bool eq = x[i] == tau;
+                    const bool sel = x[i] > tau || (eq && eq_seen < need_eq);
+                    eq_seen += eq ? 1 : 0;
+                    if (sel && cnt < P) {
+                        lk[cnt * 128 + tid] = x[i];
+                        li[cnt * 128 + tid] = c0 + i;
+                        ll[cnt * 128 + tid] = l[i];
+                        ++cnt;
+                    }
+                }
+            }
+        }
+    }
+    // NaN keys fill what is left, in id order (only rows that need it).
+    if (__any_sync(MOE_FULL_MASK, nan && cnt < kt)) {
+        for (int c0 = 0; c0 < ncols; c0 += 16) {
+            float x[16], l[16];
+            chunk_keys<MONO>(f, trow, koff, keys_in_tmem, c0, E, st, zinv, x, l, true);
+            const uint32_t cm = chunk_mask<GROUPED>(kept, c0, E, f.gsz);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                if (((cm >> i) & 1u) && nan && cnt < kt && x[i] != x[i]) {
+                    lk[cnt * 128 + tid] = x[i];
+                    li[cnt * 128 + tid] = c0 + i;
+                    ll[cnt * 128 + tid] = l[i];
+                    ++cnt;
+                }
+            }
+        }
+    }
+
+    // Order the selected by (key desc, id asc).
+    uint32_t sk[P];
+    int32_t sid[P];
+    float sl[P];
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+        const bool in = p < cnt;
+        sk[p] = in ? fkey_bits(lk[p * 128 + tid]) : 0u;
+        sid[p] = in ? li[p * 128 + tid] : 0x7fffffff;
+        sl[p] = in ? ll[p * 128 + tid] : 0.0f;
+    }
+#pragma unroll
+    for (int i = 1; i < P; ++i)
+#pragma unroll
+        for (int j = i; j > 0; --j) {
+            const bool sw = sk[j] > sk[j - 1] || (sk[j] == sk[j - 1] && sid[j] < sid[j - 1]);
+            const uint32_t tk = sw ? sk[j - 1] : sk[j];
+            const int32_t ti = sw ? sid[j - 1] : sid[j];
+            const float tl = sw ? sl[j - 1] : sl[j];
+            sk[j - 1] = sw ? sk[j] : sk[j - 1];
+            sid[j - 1] = sw ? sid[j] : sid[j - 1];
+            sl[j - 1] = sw ? sl[j] : sl[j - 1];
+            sk[j] = tk;
+            sid[j] = ti;
+            sl[j] = tl;
+        }
+
+    // Weights.
+    float sv[P];
+    float msel = -INFINITY;
+#pragma unroll
+    for (int p = 0; p < P; ++p)
+        if (p < cnt) msel = fmaxf(msel, sl[p]);
+    float sum = 0.0f;
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+        float x = 0.0f;
+        if (p < cnt) {
+            if (f.score == MOE_SCORE_SOFTMAX && !f.renorm)
+                x = expf(sl[p] - st.m) / st.z;
+            else if (f.score == MOE_SCORE_SOFTMAX || f.score == MOE_SCORE_TOPK_SOFTMAX)
+                x = expf(sl[p] - msel);
+            else if (f.score == MOE_SCORE_SIGMOID)
+                x = sigmoid_score(sl[p]);
+            else
+                x = sqrt_softplus_score(sl[p]);
+        }
+        sv[p] = x;
+        sum += x;
+    }
+    const bool norm = f.renorm || f.score == MOE_SCORE_TOPK_SOFTMAX;
+    if (valid) {
+        int32_t *orow = f.ids + row * f.k_max;
+        float *wrow = f.w + row * f.k_max;
+#pragma unroll
+        for (int p = 0; p < P; ++p)
+            if (p < f.k_max) {
+                const bool act = p < cnt;
+                orow[p] = act ? sid[p] : -1;
+                wrow[p] = act ? (norm && sum > 0.0f ? sv[p] / sum : sv[p]) * f.scale : 0.0f;
+            }
+    }
+}
+
+// MODE 0: the epilogue stores the logits.  MODE 1: it routes each row (and
+// stores the logits only if f.logits is set); MONO: keys are the logits;
+// GROUPED: a group limit applies.
+template <int MODE, int P, bool MONO = true, bool GROUPED = false>
 __global__ void __launch_bounds__(kThreads, 1)
-    gate_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
-                     const __grid_constant__ CUtensorMap tmap_w, const GemmArgs a) {
+    gate_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                const GemmArgs a, const FusedArgs f) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;  // 128-byte swizzle atoms need 1 KB alignment
     uint8_t *const gbase = smem_raw + (base - raw);
     const int S = a.stages;
-    // [stages x stage_bytes tiles][full[S]][empty[S]][tmem_full][tmem slot]
+    // [stages x stage_bytes tiles][full[S]][empty[S]][tmem_full][tmem slot][epilogue scratch]
     const uint32_t bar0 = base + (uint32_t)S * a.stage_bytes;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
     const uint32_t tmem_full_bar = bar0 + 8u * (2 * S);
     uint32_t *tmem_slot =
         reinterpret_cast<uint32_t *>(gbase + (size_t)S * a.stage_bytes + 8u * (2 * S + 1));
+    float *epi = reinterpret_cast<float *>(gbase + (size_t)S * a.stage_bytes + 256);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m0 = blockIdx.x * kBM;
@@ -230,32 +609,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp >= 4) {
         // Epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = tile rows.
         const int q = warp & 3;
-        const bool ok = mbar_wait(tmem_full_bar, 0u, a.status);
+        // TMEM loads are warp-collective: the whole warp reads or none of it.
+        const bool ok = __all_sync(MOE_FULL_MASK, mbar_wait(tmem_full_bar, 0u, a.status));
         tc_fence_after();
         const int64_t row = (int64_t)m0 + q * 32 + lane;
-        const bool vec = (a.E & 3) == 0;
-        if (ok) {
-            const int ncols = a.NC * a.BN;
-            for (int c0 = 0; c0 < ncols; c0 += 16) {
-                uint32_t r[16];
-                tmem_ld16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, r);
-                // Accumulator chunks sit side by side, so TMEM column j is expert j.
-                const int e0 = c0;
-                if (row < a.T) {
-                    float *dst = a.logits + row * a.E;
-                    if (vec && e0 + 16 <= a.E) {
+        const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16);
+        if (MODE == 0) {
+            const bool vec = (a.E & 3) == 0;
+            if (ok) {
+                const int ncols = a.NC * a.BN;
+                for (int c0 = 0; c0 < ncols; c0 += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(trow + (uint32_t)c0, r);
+                    // Accumulator chunks sit side by side, so TMEM column j is expert j.
+                    const int e0 = c0;
+                    if (row < a.T) {
+                        float *dst = a.logits + row * a.E;
+                        if (vec && e0 + 16 <= a.E) {
 #pragma unroll
-                        for (int i = 0; i < 16; i += 4)
-                            *reinterpret_cast<float4 *>(dst + e0 + i) =
-                                make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
-                                            __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
-                    } else {
+                            for (int i = 0; i < 16; i += 4)
+                                *reinterpret_cast<float4 *>(dst + e0 + i) = make_float4(
+                                    __uint_as_float(r[i]), __uint_as_float(r[i + 1]),
+                                    __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+                        } else {
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            if (e0 + i < a.E) dst[e0 + i] = __uint_as_float(r[i]);
+                            for (int i = 0; i < 16; ++i)
+                                if (e0 + i < a.E) dst[e0 + i] = __uint_as_float(r[i]);
+                        }
                     }
                 }
             }
+        } else if (ok) {
+            const int tid = q * 32 + lane;  // 0..127
+            float *gs_s = epi;              // [32][128] group scores
+            float *lk = gs_s + 32 * 128;    // [P][128] selected keys
+            int32_t *li = reinterpret_cast<int32_t *>(lk + P * 128);
+            float *ll = reinterpret_cast<float *>(li + P * 128);
+            route_epilogue<P, MONO, GROUPED>(a, f, trow, row, row < a.T, tid, gs_s, lk, li, ll);
         }
     }
 
@@ -303,22 +693,9 @@ bool make_map(CUtensorMap *m, const void *ptr, int64_t rows, int64_t cols, int b
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
-}  // namespace moe
-
-extern "C" moe_status moe_gate_gemm(const moe_bf16_t *x, const moe_bf16_t *w, float *logits,
-                                    int64_t T, int32_t d, int32_t E, int32_t *d_status,
-                                    moe_stream_t stream) {
-    using namespace moe;
-    if (T < 0 || E < 1 || E > 512 || d < 8 || d % 8 != 0) return MOE_ERR_INVALID_ARG;
-    if (T == 0) return MOE_OK;
-    if (!x || !w || !logits || !aligned16(x) || !aligned16(w)) return MOE_ERR_INVALID_ARG;
-    if (T * (int64_t)E >= (int64_t)INT32_MAX || T >= (int64_t)INT32_MAX)
-        return MOE_ERR_UNSUPPORTED;
-
-    GemmArgs a;
-    a.logits = logits;
-    a.status = d_status;
+// Shapes, stage count and shared-memory size of one launch.
+moe_status plan_gemm(int64_t T, int32_t d, int32_t E, size_t epi_bytes, GemmArgs &a,
+                     size_t &smem) {
     a.T = T;
     a.E = E;
     a.num_kb = (d + kBK - 1) / kBK;
@@ -334,7 +711,6 @@ extern "C" moe_status moe_gate_gemm(const moe_bf16_t *x, const moe_bf16_t *w, fl
     // D fp32, A and B bf16, both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
     a.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(a.BN >> 3) << 17) |
               ((uint32_t)(kBM >> 4) << 24);
-
     int dev = 0, max_smem = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
@@ -343,20 +719,120 @@ extern "C" moe_status moe_gate_gemm(const moe_bf16_t *x, const moe_bf16_t *w, fl
         return MOE_ERR_CUDA;
     }
     const int overhead = 1024 + 256;  // alignment slack + barriers and TMEM slot
-    int stages = (max_smem - overhead) / (int)a.stage_bytes;
+    int stages = (int)((max_smem - overhead - (int64_t)epi_bytes) / (int)a.stage_bytes);
     if (stages > 8) stages = 8;
     if (stages < 2) return MOE_ERR_UNSUPPORTED;
     a.stages = stages;
-    const size_t smem = (size_t)stages * a.stage_bytes + overhead;
+    smem = (size_t)stages * a.stage_bytes + overhead + epi_bytes;
+    return MOE_OK;
+}
 
+template <int MODE, int P, bool MONO = true, bool GROUPED = false>
+moe_status launch_gate(const moe_bf16_t *x, const moe_bf16_t *w, const GemmArgs &a,
+                       const FusedArgs &f, size_t smem, int32_t d, moe_stream_t stream) {
     CUtensorMap mx, mw;
-    if (!make_map(&mx, x, T, d, kBM) || !make_map(&mw, w, E, d, a.BN)) return MOE_ERR_CUDA;
-    if (cudaFuncSetAttribute(gate_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess) {
+    if (!make_map(&mx, x, a.T, d, kBM) || !make_map(&mw, w, a.E, d, a.BN)) return MOE_ERR_CUDA;
+    if (cudaFuncSetAttribute(gate_kernel<MODE, P, MONO, GROUPED>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
         cudaGetLastError();
         return MOE_ERR_CUDA;
     }
-    const unsigned grid = (unsigned)((T + kBM - 1) / kBM);
-    gate_gemm_kernel<<<grid, kThreads, smem, as_cuda(stream)>>>(mx, mw, a);
+    const unsigned grid = (unsigned)((a.T + kBM - 1) / kBM);
+    gate_kernel<MODE, P, MONO, GROUPED><<<grid, kThreads, smem, as_cuda(stream)>>>(mx, mw, a, f);
     return launch_status();
+}
+
+template <bool MONO, bool GROUPED>
+moe_status launch_fused_p(int P, const moe_bf16_t *x, const moe_bf16_t *w, const GemmArgs &a,
+                          const FusedArgs &f, size_t smem, int32_t d, moe_stream_t stream) {
+    switch (P) {
+        case 1: return launch_gate<1, 1, MONO, GROUPED>(x, w, a, f, smem, d, stream);
+        case 2: return launch_gate<1, 2, MONO, GROUPED>(x, w, a, f, smem, d, stream);
+        case 4: return launch_gate<1, 4, MONO, GROUPED>(x, w, a, f, smem, d, stream);
+        case 8: return launch_gate<1, 8, MONO, GROUPED>(x, w, a, f, smem, d, stream);
+        default: return launch_gate<1, 16, MONO, GROUPED>(x, w, a, f, smem, d, stream);
+    }
+}
+
+moe_status launch_fused(int P, bool mono, bool grouped, const moe_bf16_t *x, const moe_bf16_t *w,
+                        const GemmArgs &a, const FusedArgs &f, size_t smem, int32_t d,
+                        moe_stream_t stream) {
+    if (mono)
+        return grouped ? launch_fused_p<true, true>(P, x, w, a, f, smem, d, stream)
+                       : launch_fused_p<true, false>(P, x, w, a, f, smem, d, stream);
+    return grouped ? launch_fused_p<false, true>(P, x, w, a, f, smem, d, stream)
+                   : launch_fused_p<false, false>(P, x, w, a, f, smem, d, stream);
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" moe_status moe_gate_gemm(const moe_bf16_t *x, const moe_bf16_t *w, float *logits,
+                                    int64_t T, int32_t d, int32_t E, int32_t *d_status,
+                                    moe_stream_t stream) {
+    using namespace moe;
+    if (T < 0 || E < 1 || E > 512 || d < 8 || d % 8 != 0) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x || !w || !logits || !aligned16(x) || !aligned16(w)) return MOE_ERR_INVALID_ARG;
+    if (T * (int64_t)E >= (int64_t)INT32_MAX || T >= (int64_t)INT32_MAX)
+        return MOE_ERR_UNSUPPORTED;
+    GemmArgs a;
+    a.logits = logits;
+    a.status = d_status;
+    size_t smem = 0;
+    moe_status st = plan_gemm(T, d, E, 0, a, smem);
+    if (st != MOE_OK) return st;
+    FusedArgs f{};
+    return launch_gate<0, 1>(x, w, a, f, smem, d, stream);
+}
+
+extern "C" moe_status moe_gate_route(const moe_bf16_t *x, const moe_bf16_t *w, const float *bias,
+                                     const int32_t *k_per_token, const moe_route_params *p,
+                                     int64_t T, int32_t d, int32_t *topk_ids, float *topk_w,
+                                     float *logits, int32_t *d_status, moe_stream_t stream) {
+    using namespace moe;
+    if (!p || T < 0 || d < 8 || d % 8 != 0) return MOE_ERR_INVALID_ARG;
+    const int E = p->num_experts, G = p->n_groups;
+    if (E < 1 || E > 512 || p->k_max < 0 || p->k_max > E) return MOE_ERR_INVALID_ARG;
+    if (p->score < MOE_SCORE_SOFTMAX || p->score > MOE_SCORE_TOPK_SOFTMAX || G < 1 || E % G != 0)
+        return MOE_ERR_INVALID_ARG;
+    if (G > 32 || p->k_max > 16) return MOE_ERR_UNSUPPORTED;
+    if (G > 1 && (p->topk_groups < 1 || p->topk_groups > G || p->group_topn < 1 ||
+                  p->group_topn > 2 || p->group_topn > E / G || p->k_max > p->topk_groups * (E / G)))
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x || !w || !topk_ids || !topk_w || !aligned16(x) || !aligned16(w))
+        return MOE_ERR_INVALID_ARG;
+    if (T * (int64_t)E >= (int64_t)INT32_MAX || T >= (int64_t)INT32_MAX / 16)
+        return MOE_ERR_UNSUPPORTED;
+    int P = 1;
+    while (P < p->k_max) P *= 2;
+    GemmArgs a;
+    a.logits = logits;
+    a.status = d_status;
+    FusedArgs f;
+    f.bias = bias;
+    f.kpt = k_per_token;
+    f.ids = topk_ids;
+    f.w = topk_w;
+    f.logits = logits;
+    f.k_max = p->k_max;
+    f.score = p->score;
+    f.G = G;
+    f.TG = G > 1 ? p->topk_groups : 1;
+    f.topn = G > 1 ? p->group_topn : 1;
+    f.renorm = p->renormalize ? 1 : 0;
+    f.keys_from_scores = (bias != nullptr) || (G > 1 && f.topn > 1);
+    f.gsz = E / G;
+    f.scale = p->route_scale;
+    const size_t epi = (size_t)32 * 128 * 4 + (size_t)P * 128 * 12;
+    size_t smem = 0;
+    moe_status st = plan_gemm(T, d, E, epi, a, smem);
+    if (st != MOE_OK) return st;
+    // Score keys keep a copy in spare TMEM columns when the accumulator uses at
+    // most half of the 512 columns.
+    if (f.keys_from_scores && a.NC * a.BN <= 256) a.tmem_cols = 512;
+    const bool mono = !f.keys_from_scores;
+    const bool grouped = G > 1;
+    return launch_fused(P, mono, grouped, x, w, a, f, smem, d, stream);
 }

@@ -19,6 +19,10 @@ gives the expert counts, k, scoring and shared experts of the families;
                  one shared expert; logits ~N(0,1), 10% of rows +3 on 4 hot experts
   gptoss_top4    T=262144, d=2880, E=128, k=4, gpt-oss (softmax over the 4
                  selected logits); logits as llama4_top1
+  llama4_top1_capacity
+                 llama4_top1 with a Switch-style capacity (factor 1.0: each
+                 expert keeps at most T/E = 2048 tokens, the skewed hot experts
+                 drop the rest) and expert blocks padded to 128 rows
 Seeds: 1000 * workload index + tensor index.  bf16 tensors are drawn in fp32
 and rounded to bf16 (round to nearest even).
 """
@@ -53,6 +57,19 @@ class Workload:
     combine: bool = True           # the path ends at combine (else at permute)
     hash_vocab: int = 0            # > 0: a hash-routed layer is part of the workload
     w_std: float = 0.02
+    capacity_factor: float = 0.0   # > 0: per-expert capacity ceil(cf * T * k / E)
+    pad: int = 1                   # expert blocks padded to a multiple of this many rows
+
+    @property
+    def limited(self) -> bool:
+        """Dispatch with a capacity and/or padded expert blocks."""
+        return self.capacity_factor > 0 or self.pad > 1
+
+    @property
+    def capacity(self) -> int:
+        if self.capacity_factor <= 0:
+            return 0
+        return max(1, math.ceil(self.capacity_factor * self.T * self.k_max / self.E))
 
     def scaled(self, T: int) -> "Workload":
         """Same workload with another token count (smaller parity cases)."""
@@ -73,6 +90,9 @@ WORKLOADS = {
                  gate=False, renormalize=False, shared=True, skew=True),
         Workload("gptoss_top4", 6, T=262144, d=2880, E=128, k_max=4, score="topk_softmax",
                  gate=False, skew=True),
+        Workload("llama4_top1_capacity", 7, T=262144, d=5120, E=128, k_max=1, score="sigmoid",
+                 gate=False, renormalize=False, shared=True, skew=True, capacity_factor=1.0,
+                 pad=128),
     ]
 }
 
@@ -107,6 +127,17 @@ def num_assignments(wl: Workload, kpt) -> int:
     return int(kpt.sum().item()) if kpt is not None else wl.T * wl.k_max
 
 
+def expert_rows(wl: Workload, kpt) -> int:
+    """Rows of the expert-ordered buffers (xs, y): N, or with a capacity and
+    padded blocks the most they can need, min(N, E * capacity) + E * (pad - 1)."""
+    n = num_assignments(wl, kpt)
+    if not wl.limited:
+        return n
+    if wl.capacity:
+        n = min(n, wl.E * wl.capacity)
+    return n + wl.E * (wl.pad - 1)
+
+
 def make_inputs(wl: Workload, device="cuda", *, with_y=True, with_x=True,
                 seed_offset: int = 0) -> dict:
     """All seeded inputs of one workload on ``device``.
@@ -136,7 +167,7 @@ def make_inputs(wl: Workload, device="cuda", *, with_y=True, with_x=True,
         out["bias"] = (b * 0.2 - 0.1).contiguous()
     out["k_per_token"] = k_per_token(wl, device, s + 3)
     if with_y and wl.combine:
-        n = num_assignments(wl, out["k_per_token"])
+        n = expert_rows(wl, out["k_per_token"])
         out["y"] = normal_bf16((n, wl.d), 1.0, device, s + 4)
     if wl.shared and wl.combine:
         out["shared"] = normal_bf16((wl.T, wl.d), 1.0, device, s + 7)
