@@ -110,9 +110,26 @@ def stage_bytes(wl, n_assign: int, fused: bool = False, limited=None) -> dict:
                       + (E * 4 if wl.bias else 0))
     b["dispatch"] = T * k * 4 + n_assign * 4 + T * k * 4 + 8 * E + pad_rows * 4
     b["permute"] = t_read * d * 2 + n_assign * d * 2 + T * k * 4
+    if wl.ffn_dim and wl.pad % 128 == 0:  # the experts' FFN on the kept rows
+        F = wl.ffn_dim
+        bias = wl.ffn_act == "swiglu_oai"
+        b["expert_gate_up"] = (n_assign * d * 2 + 2 * E * F * d * 2 + n_assign * F * 2
+                               + (2 * E * F * 4 if bias else 0))
+        b["expert_down"] = n_assign * F * 2 + E * d * F * 2 + n_assign * d * 2 + (E * d * 4 if bias else 0)
     if wl.combine:
         b["combine"] = n_assign * d * 2 + T * d * 2 + (T * d * 2 if wl.shared else 0) + 8 * T * k
     return b
+
+
+def stage_flops(wl, n_assign: int) -> dict:
+    """Algorithmic FLOPs of the tensor-core stages (padding rows excluded)."""
+    f = {}
+    if wl.gate:
+        f["gate_route"] = f["gate_gemm"] = 2.0 * wl.T * wl.E * wl.d
+    if wl.ffn_dim and wl.pad % 128 == 0:
+        f["expert_gate_up"] = 2.0 * n_assign * 2 * wl.ffn_dim * wl.d
+        f["expert_down"] = 2.0 * n_assign * wl.ffn_dim * wl.d
+    return f
 
 
 def load_peaks():
@@ -203,9 +220,10 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- oracle chain
-def oracle_inputs(wl, inp: dict, n_tokens: int) -> dict:
+def oracle_inputs(wl, inp: dict, n_tokens: int, experts=None) -> dict:
     """Host copies of the first n_tokens tokens of a workload's inputs, with
-    expert outputs for the sample's own assignments."""
+    expert outputs for the sample's own assignments (or, given the experts'
+    weights, host copies of those)."""
     from token_dispatch_moe_b200.workloads import normal_bf16
 
     def bits(t):
@@ -222,12 +240,18 @@ def oracle_inputs(wl, inp: dict, n_tokens: int) -> dict:
     n += wl.E * (wl.pad - 1)  # padded expert blocks
     h["y"] = bits(normal_bf16((max(n, 1), wl.d), 1.0, "cpu", 1000 * wl.index + 44))
     h["shared"] = bits(inp["shared"][:n_tokens]) if inp["shared"] is not None else None
+    h["experts"] = None
+    if experts is not None:
+        h["experts"] = {k: (None if v is None else
+                            (bits(v) if v.dtype == torch.bfloat16 else v.cpu().numpy()))
+                        for k, v in experts.items()}
     return h
 
 
 def oracle_chain(wl, h: dict) -> None:
     """The path computed by the fp64 CPU oracle (single thread): gate, route,
-    dispatch, permute, combine, on the sample held in h."""
+    dispatch, permute, [the experts' FFN when h holds their weights], combine,
+    on the sample held in h."""
     import oracle
     score = {"softmax": oracle.SOFTMAX, "sigmoid": oracle.SIGMOID,
              "sqrt_softplus": oracle.SQRT_SOFTPLUS, "topk_softmax": oracle.TOPK_SOFTMAX}[wl.score]
@@ -241,16 +265,28 @@ def oracle_chain(wl, h: dict) -> None:
     else:
         dsp = oracle.dispatch(r["ids"], wl.E)
     n = int(dsp["offsets"][-1])
-    oracle.permute(h["x"], dsp["dest_pos"], n)
+    xs = oracle.permute(h["x"], dsp["dest_pos"], n)
+    y = h["y"]
+    if h.get("experts") is not None:
+        ex = h["experts"]
+        act = oracle.SWIGLU_OAI if wl.ffn_act == "swiglu_oai" else oracle.SWIGLU
+        rows = np.nonzero(dsp["sorted_token"] >= 0)[0]
+        hid = np.zeros((max(n, 1), wl.ffn_dim), np.uint16)
+        hv = oracle.expert_gate_up(xs, dsp["offsets"], ex["w1"], ex["w3"], rows, act=act,
+                                   b1=ex["b1"], b3=ex["b3"])
+        hid[rows] = torch.from_numpy(hv).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        yv = oracle.expert_down(hid, dsp["offsets"], ex["w2"], rows, b2=ex["b2"])
+        y = np.zeros((max(n, 1), wl.d), np.uint16)
+        y[rows] = torch.from_numpy(yv).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     if wl.combine:
-        oracle.combine(h["y"][:max(n, 1)], r["w"].astype(np.float32), dsp["dest_pos"],
+        oracle.combine(y[:max(n, 1)], r["w"].astype(np.float32), dsp["dest_pos"],
                        h["shared"], want_mag=False)
 
 
-def oracle_sample_size(wl, inp, budget_s: float) -> int:
+def oracle_sample_size(wl, inp, budget_s: float, experts=None) -> int:
     """Tokens of CPU work that take about budget_s seconds (calibrated on a small run)."""
-    n0 = min(64, wl.T)
-    h = oracle_inputs(wl, inp, n0)
+    n0 = min(64 if experts is None else 8, wl.T)
+    h = oracle_inputs(wl, inp, n0, experts)
     t0 = time.perf_counter()
     oracle_chain(wl, h)
     per_token = (time.perf_counter() - t0) / n0
@@ -277,7 +313,12 @@ def run_ours(args):
     wl = WORKLOADS[args.workload]
     if args.tokens:
         wl = wl.scaled(args.tokens)
-    inp = make_inputs(wl, device, seed_offset=rank_seed_offset(rank))
+    experts = None
+    if args.ffn:
+        from token_dispatch_moe_b200.workloads import make_expert_weights
+        wl = wl.with_ffn()
+        experts = make_expert_weights(wl, device, seed_offset=rank_seed_offset(rank))
+    inp = make_inputs(wl, device, with_y=experts is None, seed_offset=rank_seed_offset(rank))
     n_assign = num_assignments(wl, inp["k_per_token"])
     path = RouterDispatch(wl, device, fused=False if args.separate else (True if args.fused else None))
     stream = torch.cuda.current_stream(device)
@@ -311,8 +352,15 @@ def run_ours(args):
         boundary()
         path.permute(inp["x"])
         boundary()
+        y = inp["y"]
+        if experts is not None:
+            path.expert_gate_up(experts)
+            boundary()
+            path.expert_down(experts)
+            boundary()
+            y = path.y
         if wl.combine:
-            path.combine(inp["y"], inp["shared"])
+            path.combine(y, inp["shared"])
             boundary()
 
     for _ in range(args.warmup):
@@ -399,28 +447,37 @@ def run_ours(args):
         gbs = bytes_per[n] / (stage_ms[n] / 1e3) / 1e9
         stages[n] = {"us": round(stage_ms[n] * 1e3, 2), "bytes": bytes_per[n],
                      "GB_s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4)}
-    gname = "gate_route" if path.fused else "gate_gemm"
-    if wl.gate:
-        flops = 2.0 * wl.T * wl.E * wl.d
-        stages[gname]["TFLOP_s"] = round(flops / (stage_ms[gname] / 1e3) / 1e12, 1)
-        stages[gname]["frac_tensor"] = round(stages[gname]["TFLOP_s"] / tf_sust, 4)
+    kept = limited[0] if limited else n_assign
+    flops = stage_flops(wl, kept)
+    for n in names:
+        if n in flops:
+            stages[n]["TFLOP_s"] = round(flops[n] / (stage_ms[n] / 1e3) / 1e12, 1)
+            stages[n]["frac_tensor"] = round(stages[n]["TFLOP_s"] / tf_sust, 4)
     dom = max(stage_ms, key=stage_ms.get)
-    achieved = bytes_per[dom] / (stage_ms[dom] / 1e3) / 1e9
-    roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
-                "unit": "GB/s", "frac": round(achieved / hbm, 4),
-                "traffic": recorded_traffic(wl.name, dom),
-                "algorithmic_bytes": bytes_per[dom], "peak_source": peak_kind}
+    if dom.startswith("expert_"):  # a dense contraction: bound by the tensor pipe
+        achieved = flops[dom] / (stage_ms[dom] / 1e3) / 1e12
+        roofline = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1),
+                    "peak": tf_sust, "unit": "TFLOP/s", "frac": round(achieved / tf_sust, 4),
+                    "traffic": recorded_traffic(wl.name + "+ffn", dom),
+                    "algorithmic_flops": flops[dom], "peak_source": peak_kind + " (sustained)"}
+    else:
+        achieved = bytes_per[dom] / (stage_ms[dom] / 1e3) / 1e9
+        roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
+                    "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                    "traffic": recorded_traffic(wl.name, dom),
+                    "algorithmic_bytes": bytes_per[dom], "peak_source": peak_kind}
 
     e2e = None
     if not args.no_e2e:
-        e2e = measure_e2e(wl, inp, path, device, stream, min(K, args.e2e_steps), world)
+        e2e = measure_e2e(wl, inp, path, device, stream, min(K, args.e2e_steps), world, experts)
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_max, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
         "data": "synthetic",
-        "config": {"workload": wl.name if not args.tokens else f"{wl.name}@T={wl.T}",
+        "config": {"workload": (wl.name + ("+ffn" if experts is not None else "")
+                                + (f"@T={wl.T}" if args.tokens else "")),
                    "tokens_per_gpu": wl.T, "hidden": wl.d, "experts": wl.E,
                    "k": (f"{'/'.join(map(str, wl.k_choices))} per {wl.segment}-token request"
                          if wl.k_choices else wl.k_max),
@@ -434,17 +491,18 @@ def run_ours(args):
                        "pad_rows_to": wl.pad, "kept_slots": limited[0],
                        "dropped_slots": n_assign - limited[0]} if limited else {})},
         "roofline": roofline, "stages": stages, "clocks": clk.summary(),
-        "gpu_launches": chain_launches(wl, path.fused) * K, "e2e": e2e,
+        "gpu_launches": (chain_launches(wl, path.fused) + (2 if experts is not None else 0)) * K,
+        "e2e": e2e,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(wl, inp, args.cpu_budget)
+        result["cpu_baseline"] = cpu_baseline(wl, inp, args.cpu_budget, experts)
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
 
 
-def measure_e2e(wl, inp, path, device, stream, steps, world):
+def measure_e2e(wl, inp, path, device, stream, steps, world, experts=None):
     """Same metric through the C ABI with host buffers: each step copies its
     inputs from pinned host memory, runs the chain and copies the result back."""
     names = [k for k in ("x", "w", "logits", "bias", "k_per_token", "y", "shared") if
@@ -461,7 +519,7 @@ def measure_e2e(wl, inp, path, device, stream, steps, world):
     def one():
         for k in names:
             dev[k].copy_(host[k], non_blocking=True)
-        path.run(full)
+        path.run(full, experts=experts)
         out_host.copy_(result_dev, non_blocking=True)
 
     one()
@@ -482,9 +540,9 @@ def measure_e2e(wl, inp, path, device, stream, steps, world):
             "steps": steps}
 
 
-def cpu_baseline(wl, inp, budget_s: float) -> dict:
-    n = oracle_sample_size(wl, inp, budget_s)
-    h = oracle_inputs(wl, inp, n)
+def cpu_baseline(wl, inp, budget_s: float, experts=None) -> dict:
+    n = oracle_sample_size(wl, inp, budget_s, experts)
+    h = oracle_inputs(wl, inp, n, experts)
     t0 = time.perf_counter()
     oracle_chain(wl, h)
     dt = time.perf_counter() - t0
@@ -498,13 +556,18 @@ def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
         return  # the CPU oracle runs once, on rank 0
-    from token_dispatch_moe_b200.workloads import WORKLOADS, make_inputs
+    from token_dispatch_moe_b200.workloads import WORKLOADS, make_expert_weights, make_inputs
     wl = WORKLOADS[args.workload]
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    inp = make_inputs(wl, dev, with_y=False)
+    experts = None
+    if args.ffn:
+        wl = wl.with_ffn()
+        experts = make_expert_weights(wl, dev)
+    inp = make_inputs(wl, dev, with_y=experts is None)
     total_budget = args.cpu_budget
-    per_step = oracle_sample_size(wl, inp, total_budget / max(1, args.steps + args.warmup))
-    h = oracle_inputs(wl, inp, per_step)
+    per_step = oracle_sample_size(wl, inp, total_budget / max(1, args.steps + args.warmup),
+                                  experts)
+    h = oracle_inputs(wl, inp, per_step, experts)
     for _ in range(args.warmup):
         oracle_chain(wl, h)
     t0 = time.perf_counter()
@@ -516,7 +579,8 @@ def run_reference(args):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "tokens_per_step": per_step,
+            "config": {"workload": wl.name + ("+ffn" if experts is not None else ""),
+                       "tokens_per_step": per_step,
                        "parallelism": "single host core"},
             "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": 1,
                              "kind": "oracle",
@@ -539,6 +603,9 @@ def main(argv=None):
                     help="run the gate GEMM and the route as two kernels instead of one")
     ap.add_argument("--fused", action="store_true",
                     help="route inside the gate GEMM even where two kernels are faster")
+    ap.add_argument("--ffn", action="store_true",
+                    help="run the experts' SwiGLU FFN (synthetic weights) on the permuted rows "
+                         "instead of reading synthetic expert outputs")
     ap.add_argument("--eager", action="store_true",
                     help="launch from the host every step instead of replaying a CUDA graph")
     ap.add_argument("--no-e2e", action="store_true")

@@ -130,6 +130,24 @@ moe_status moe_route(const float *logits, const float *bias, const int32_t *k_pe
                      float *topk_w, int32_t *d_status, moe_stream_t stream);
 
 /*
+ * moe_route_grouped -- grouped top-k ("Crate ferrox_moe", Functions,
+ * route_top_k_grouped): the E experts form params->n_groups contiguous
+ * groups; each group keeps its k_per_group best experts by score (the same
+ * score function as moe_route), and of those candidates the params->k_max best
+ * are selected, in descending score order, ties to the lower id.  Weights as
+ * moe_route (score of the expert, renormalize, route_scale; gpt-oss: softmax
+ * over the selected logits).  No bias and no per-token k: the page gives the
+ * rule without them.  params->topk_groups and group_topn are ignored.
+ * logits [T][E] fp32 (4-byte aligned); topk_ids, topk_w [T][k_max].
+ * Limits: E <= 512, E % n_groups == 0, 1 <= k_per_group <= E/n_groups,
+ * k_max <= min(32, n_groups * k_per_group).  NaN logits rank lowest and report
+ * MOE_ERR_NAN_LOGIT.
+ */
+moe_status moe_route_grouped(const float *logits, const moe_route_params *params,
+                             int32_t k_per_group, int64_t T, int32_t *topk_ids, float *topk_w,
+                             int32_t *d_status, moe_stream_t stream);
+
+/*
  * moe_gate_route -- moe_gate_gemm and moe_route in one kernel (the gate linear
  * and the router are one function in "DeepSeek-V3.2-Exp - Select experts",
  * gate forward).  Same inputs, outputs and status rules as the two calls in a
@@ -334,6 +352,47 @@ moe_status moe_ep_combine(moe_bf16_t *const *peer_y, const int32_t *dest_rank,
                           const int32_t *dest_row, const float *topk_w, const moe_bf16_t *shared,
                           int32_t G, int64_t recv_capacity, int64_t T, int32_t k_max, int32_t d,
                           moe_bf16_t *out, int32_t *d_status, moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Routed experts' FFN over the expert-ordered rows ("Crate ferrox_moe",
+ * Functions: run_expert, run_expert_oai, swiglu_oai; Constants:
+ * SWIGLU_OAI_ALPHA = 1.702, SWIGLU_OAI_LIMIT = 7.0).  Two grouped GEMMs on
+ * tcgen05 tensor cores; row r belongs to the expert e whose block
+ * [offsets[e], offsets[e+1]) holds it, and the blocks must start on multiples
+ * of 128 rows (moe_dispatch_limited with pad = 128 writes such offsets; rows
+ * of a block past the expert's own tokens are padding and give padding).
+ * The page names the clamped SwiGLU and its constants but not its formula;
+ * the reading here is the published gpt-oss one:
+ *   MOE_ACT_SWIGLU:     act(g, u) = g * sigmoid(g) * u
+ *   MOE_ACT_SWIGLU_OAI: g' = min(g, 7), u' = clamp(u, -7, 7),
+ *                       act(g, u) = g' * sigmoid(1.702 * g') * (u' + 1)
+ * ------------------------------------------------------------------------ */
+typedef enum { MOE_ACT_SWIGLU = 0, MOE_ACT_SWIGLU_OAI = 1 } moe_activation;
+
+/*
+ * moe_expert_gate_up -- h[r] = bf16( act(xs[r] . W1[e]^T + b1[e],
+ *                                        xs[r] . W3[e]^T + b3[e]) )
+ * xs [rows][d] bf16; w1, w3 [E][F][d] bf16 (row f of expert e is the weight
+ * vector of output feature f, K-major); b1, b3 [E][F] fp32 or NULL;
+ * h [rows][F] bf16.  fp32 accumulation, activation in fp32, one rounding.
+ * d, F multiples of 16; E <= 4096; rows/128 <= 65535; xs, w1, w3, h 16-byte
+ * aligned.  Offsets not 128-aligned, or offsets[E] > rows, report
+ * MOE_ERR_DEVICE_INDEX and leave the affected tiles unwritten.
+ */
+moe_status moe_expert_gate_up(const moe_bf16_t *xs, const int32_t *offsets, const moe_bf16_t *w1,
+                              const moe_bf16_t *w3, const float *b1, const float *b3, int32_t E,
+                              int32_t d, int32_t F, int64_t rows, int32_t act, moe_bf16_t *h,
+                              int32_t *d_status, moe_stream_t stream);
+
+/*
+ * moe_expert_down -- y[r] = bf16( h[r] . W2[e]^T + b2[e] )
+ * h [rows][F] bf16; w2 [E][d][F] bf16; b2 [E][d] fp32 or NULL; y [rows][d]
+ * bf16 (the expert outputs moe_combine reads).  Limits and status as
+ * moe_expert_gate_up.
+ */
+moe_status moe_expert_down(const moe_bf16_t *h, const int32_t *offsets, const moe_bf16_t *w2,
+                           const float *b2, int32_t E, int32_t d, int32_t F, int64_t rows,
+                           moe_bf16_t *y, int32_t *d_status, moe_stream_t stream);
 
 #ifdef __cplusplus
 }

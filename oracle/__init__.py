@@ -82,6 +82,10 @@ def _bind(lib):
     lib.oracle_dispatch_limited.restype = ctypes.c_int
     lib.oracle_route_grouped.argtypes = [P, i64, i32, i32, i32, i32, i32, i32, f64, P, P, P]
     lib.oracle_route_grouped.restype = ctypes.c_int
+    lib.oracle_expert_gate_up.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, P, i64, P, P, P]
+    lib.oracle_expert_gate_up.restype = ctypes.c_int
+    lib.oracle_expert_down.argtypes = [P, P, P, P, i32, i32, i32, P, i64, P]
+    lib.oracle_expert_down.restype = ctypes.c_int
     lib.oracle_ep_layout.argtypes = [P, i32, i64, i32, i32, P, P, P]
     lib.oracle_ep_layout.restype = ctypes.c_int
     lib.oracle_permute.argtypes = [P, P, i64, i32, i32, P]
@@ -274,6 +278,46 @@ def ep_combine(y_bits_per_rank, w_all, dest_rank, dest_row, shared_all_bits=None
                             None if shared_all_bits is None else shared_all_bits[r],
                             want_mag=want_mag))
     return outs
+
+
+SWIGLU, SWIGLU_OAI = 0, 1
+
+
+def expert_gate_up(xs_bits, offsets, w1_bits, w3_bits, rows, *, act=SWIGLU, b1=None, b3=None,
+                   want_pre=False):
+    """h rows (fp64, unrounded) of the experts' gate/up step for the listed rows."""
+    xs = _c(xs_bits, np.uint16)
+    off = _c(offsets, np.int32)
+    w1 = _c(w1_bits, np.uint16)
+    w3 = _c(w3_bits, np.uint16)
+    E, F, d = w1.shape
+    r = _c(rows, np.int64)
+    h = np.empty((r.size, F), np.float64)
+    g = np.empty((r.size, F), np.float64) if want_pre else None
+    u = np.empty((r.size, F), np.float64) if want_pre else None
+    bb1 = None if b1 is None else _c(b1, np.float32)
+    bb3 = None if b3 is None else _c(b3, np.float32)
+    st = _load().oracle_expert_gate_up(_p(xs), _p(off), _p(w1), _p(w3), _p(bb1), _p(bb3), E, d, F,
+                                       act, _p(r), r.size, _p(h), _p(g), _p(u))
+    if st != OK:
+        raise ValueError("oracle_expert_gate_up: a row lies in no expert block")
+    return (h, g, u) if want_pre else h
+
+
+def expert_down(h_bits, offsets, w2_bits, rows, *, b2=None):
+    """y rows (fp64) of the experts' down projection for the listed rows of h."""
+    hb = _c(h_bits, np.uint16)
+    off = _c(offsets, np.int32)
+    w2 = _c(w2_bits, np.uint16)
+    E, d, F = w2.shape
+    r = _c(rows, np.int64)
+    y = np.empty((r.size, d), np.float64)
+    bb2 = None if b2 is None else _c(b2, np.float32)
+    st = _load().oracle_expert_down(_p(hb), _p(off), _p(w2), _p(bb2), E, d, F, _p(r), r.size,
+                                    _p(y))
+    if st != OK:
+        raise ValueError("oracle_expert_down: a row lies in no expert block")
+    return y
 
 
 def permute(x_bits, dest_pos, n_rows: int) -> np.ndarray:

@@ -477,6 +477,84 @@ int oracle_ep_layout(const int32_t *ids_all, int32_t G, int64_t T, int32_t k_max
     return status;
 }
 
+/* ------------------------------------------------------- expert FFN ---- */
+/* [FX] run_expert / run_expert_oai / swiglu_oai: an expert's FFN is gate and
+ * up projections of the hidden row, a gated activation, and a down
+ * projection (gpt-oss: a bias on each product, the clamped SwiGLU with
+ * alpha = 1.702 and limit 7.0).  The page gives the constants but not the
+ * clamped formula; the reading is the published gpt-oss one:
+ *   act = 0 (SwiGLU):  g * sigmoid(g) * u
+ *   act = 1 (gpt-oss): g' = min(g, 7), u' = clamp(u, -7, 7),
+ *                      g' * sigmoid(1.702 g') * (u' + 1)
+ * Row r belongs to expert e with offsets[e] <= r < offsets[e+1].  Returns -1
+ * for a row outside every block. */
+#define ORACLE_OAI_ALPHA 1.702
+#define ORACLE_OAI_LIMIT 7.0
+
+static double oracle_act(int32_t act, double g, double u) {
+    if (act == 1) {
+        double gc = g < ORACLE_OAI_LIMIT ? g : ORACLE_OAI_LIMIT;
+        double uc = u < -ORACLE_OAI_LIMIT ? -ORACLE_OAI_LIMIT : (u > ORACLE_OAI_LIMIT ? ORACLE_OAI_LIMIT : u);
+        return gc * (1.0 / (1.0 + exp(-ORACLE_OAI_ALPHA * gc))) * (uc + 1.0);
+    }
+    return g * (1.0 / (1.0 + exp(-g))) * u;
+}
+
+static int32_t row_expert(const int32_t *offsets, int32_t E, int64_t r) {
+    for (int32_t e = 0; e < E; ++e)
+        if (offsets[e] <= r && r < offsets[e + 1]) return e;
+    return -1;
+}
+
+/* h[i][f] (fp64, before any rounding) for the listed rows of xs; g_out and
+ * u_out (optional) receive the two pre-activation products. */
+int oracle_expert_gate_up(const uint16_t *xs, const int32_t *offsets, const uint16_t *w1,
+                          const uint16_t *w3, const float *b1, const float *b3, int32_t E,
+                          int32_t d, int32_t F, int32_t act, const int64_t *rows, int64_t nrows,
+                          double *h, double *g_out, double *u_out) {
+    for (int64_t i = 0; i < nrows; ++i) {
+        const int32_t e = row_expert(offsets, E, rows[i]);
+        if (e < 0) return ORACLE_ERR_INDEX;
+        const uint16_t *x = xs + rows[i] * (int64_t)d;
+        for (int32_t f = 0; f < F; ++f) {
+            const uint16_t *r1 = w1 + ((int64_t)e * F + f) * d;
+            const uint16_t *r3 = w3 + ((int64_t)e * F + f) * d;
+            double g = 0.0, u = 0.0;
+            for (int32_t k = 0; k < d; ++k) {
+                g += oracle_bf16_to_double(x[k]) * oracle_bf16_to_double(r1[k]);
+                u += oracle_bf16_to_double(x[k]) * oracle_bf16_to_double(r3[k]);
+            }
+            if (b1) g += (double)b1[(int64_t)e * F + f];
+            if (b3) u += (double)b3[(int64_t)e * F + f];
+            h[i * F + f] = oracle_act(act, g, u);
+            if (g_out) g_out[i * F + f] = g;
+            if (u_out) u_out[i * F + f] = u;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* y[i][c] = sum_f h[row][f] * W2[e][c][f] + b2[e][c] (fp64) for the listed rows
+ * of h (bf16 bits, e.g. the device's h). */
+int oracle_expert_down(const uint16_t *h, const int32_t *offsets, const uint16_t *w2,
+                       const float *b2, int32_t E, int32_t d, int32_t F, const int64_t *rows,
+                       int64_t nrows, double *y) {
+    for (int64_t i = 0; i < nrows; ++i) {
+        const int32_t e = row_expert(offsets, E, rows[i]);
+        if (e < 0) return ORACLE_ERR_INDEX;
+        const uint16_t *hr = h + rows[i] * (int64_t)F;
+        for (int32_t c = 0; c < d; ++c) {
+            const uint16_t *wr = w2 + ((int64_t)e * d + c) * F;
+            double acc = 0.0;
+            for (int32_t f = 0; f < F; ++f)
+                acc += oracle_bf16_to_double(hr[f]) * oracle_bf16_to_double(wr[f]);
+            if (b2) acc += (double)b2[(int64_t)e * d + c];
+            y[i * d + c] = acc;
+        }
+    }
+    return ORACLE_OK;
+}
+
 /* ------------------------------------------------------------- permute ---- */
 /* xs[dest_pos[t][j]] = x[t] for every filled slot: a bit-exact row copy. */
 void oracle_permute(const uint16_t *x, const int32_t *dest_pos, int64_t T, int32_t k_max,

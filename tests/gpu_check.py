@@ -166,3 +166,41 @@ def check_combine(out_gpu, y, topk_w, dest_pos, shared=None, tokens=None) -> flo
     worst = float(ratio.max()) if ratio.size else 0.0
     assert np.all(ratio <= COMBINE_RTOL), f"combine out of tolerance, worst {worst}"
     return worst
+
+
+# ----------------------------------------------------------- expert FFN
+# h  |g - o| <= 2^-8 |o| + (|u| + 1) dg + (|g| + 1) du, where dg, du =
+#    1e-5 * sum_k |x_k w_k| bound the fp32 accumulation of the two products
+#    (the activation's derivatives are below |u|+1 and |g|+1), and 2^-8 is one
+#    bf16 rounding of h;
+# y  |g - o| <= 2^-8 |o| + 1e-5 * sum_f |h_f w2_f|, fed with the device's h.
+def abs_bits(b):
+    return b & np.uint16(0x7FFF)
+
+
+def _np(t):
+    return None if t is None else t.cpu().numpy()
+
+
+def check_expert_h(h, xs, offsets, w1, w3, b1, b3, act, rows):
+    off = offsets.cpu().numpy()
+    xb, w1b, w3b = bits(xs), bits(w1), bits(w3)
+    o, g, u = oracle.expert_gate_up(xb, off, w1b, w3b, rows, act=act, b1=_np(b1), b3=_np(b3),
+                                    want_pre=True)
+    _, ga, ua = oracle.expert_gate_up(abs_bits(xb), off, abs_bits(w1b), abs_bits(w3b), rows,
+                                      want_pre=True)
+    got = bits_to_f64(bits(h)[rows])
+    tol = 2.0 ** -8 * np.abs(o) + (np.abs(u) + 1) * 1e-5 * ga + (np.abs(g) + 1) * 1e-5 * ua
+    bad = np.argwhere(np.abs(got - o) > tol)
+    assert bad.size == 0, f"h: {len(bad)} values out of tolerance, first {bad[:5].tolist()}"
+
+
+def check_expert_y(y, h, offsets, w2, b2, rows):
+    off = offsets.cpu().numpy()
+    hb, w2b = bits(h), bits(w2)
+    o = oracle.expert_down(hb, off, w2b, rows, b2=_np(b2))
+    mag = oracle.expert_down(abs_bits(hb), off, abs_bits(w2b), rows)
+    got = bits_to_f64(bits(y)[rows])
+    tol = 2.0 ** -8 * np.abs(o) + 1e-5 * mag
+    bad = np.argwhere(np.abs(got - o) > tol)
+    assert bad.size == 0, f"y: {len(bad)} values out of tolerance, first {bad[:5].tolist()}"

@@ -524,6 +524,64 @@ def pin_ep_layout():
         assert np.array_equal(outs[g], _bits_to_f64(x[g]))
 
 
+def pin_expert_ffn():
+    sig = lambda v: 1.0 / (1.0 + math.exp(-v))  # noqa: E731
+    # Activation closed forms through 1-wide experts: xs = [1], so g = w1, u = w3.
+    off = np.array([0, 1], np.int32)
+    one = _bf16_bits_from_f32(np.array([[1.0] + [0.0] * 15], np.float32))
+    for act, g, u, want in ((oracle.SWIGLU, 0.0, 5.0, 0.0),
+                            (oracle.SWIGLU, 2.0, 3.0, 2.0 * sig(2.0) * 3.0),
+                            (oracle.SWIGLU_OAI, 10.0, 2.0, 7.0 * sig(1.702 * 7.0) * 3.0),
+                            (oracle.SWIGLU_OAI, 3.0, -20.0, 3.0 * sig(1.702 * 3.0) * -6.0),
+                            (oracle.SWIGLU_OAI, -20.0, 1.0, -20.0 * sig(-1.702 * 20.0) * 2.0),
+                            (oracle.SWIGLU_OAI, 1.0, -1.0, 0.0)):
+        w1 = _bf16_bits_from_f32(np.array([[[g] + [0.0] * 15]], np.float32))
+        w3 = _bf16_bits_from_f32(np.array([[[u] + [0.0] * 15]], np.float32))
+        h = oracle.expert_gate_up(one, off, w1, w3, [0], act=act)
+        assert abs(h[0, 0] - want) <= 1e-14 * max(1.0, abs(want)), (act, g, u, h[0, 0], want)
+    # Integer-valued operands: the products are exact, so g, u and y equal an
+    # integer matmul; each row uses the weights of the block holding it.
+    rng = np.random.default_rng(67)
+    E, d, F = 3, 16, 8
+    offsets = np.array([0, 4, 4, 9], np.int32)  # expert 1 holds no rows
+    R = 9
+    xi = rng.integers(-3, 4, size=(R, d))
+    w1i = rng.integers(-2, 3, size=(E, F, d))
+    w3i = rng.integers(-2, 3, size=(E, F, d))
+    w2i = rng.integers(-2, 3, size=(E, d, F))
+    b1 = rng.integers(-4, 5, size=(E, F)).astype(np.float32)
+    b3 = rng.integers(-4, 5, size=(E, F)).astype(np.float32)
+    b2 = rng.integers(-4, 5, size=(E, d)).astype(np.float32)
+    bits = lambda a: _bf16_bits_from_f32(a.astype(np.float32))  # noqa: E731
+    rows = np.arange(R)
+    for act in (oracle.SWIGLU, oracle.SWIGLU_OAI):
+        h, g, u = oracle.expert_gate_up(bits(xi), offsets, bits(w1i), bits(w3i), rows, act=act,
+                                        b1=b1, b3=b3, want_pre=True)
+        for r in rows:
+            e = 0 if r < 4 else 2
+            gi = w1i[e] @ xi[r] + b1[e]
+            ui = w3i[e] @ xi[r] + b3[e]
+            assert np.array_equal(g[r], gi) and np.array_equal(u[r], ui)
+            for f in range(F):
+                gv, uv = float(gi[f]), float(ui[f])
+                if act == oracle.SWIGLU:
+                    want = gv * sig(gv) * uv
+                else:
+                    gc, uc = min(gv, 7.0), min(max(uv, -7.0), 7.0)
+                    want = gc * sig(1.702 * gc) * (uc + 1.0)
+                assert abs(h[r, f] - want) <= 1e-12 * max(1.0, abs(want))
+    hi = rng.integers(-3, 4, size=(R, F))
+    y = oracle.expert_down(bits(hi), offsets, bits(w2i), rows, b2=b2)
+    for r in rows:
+        e = 0 if r < 4 else 2
+        assert np.array_equal(y[r], w2i[e] @ hi[r] + b2[e])
+    try:
+        oracle.expert_down(bits(hi), offsets, bits(w2i), [R])  # row past the last block
+        raise AssertionError("a row outside every block must be refused")
+    except ValueError:
+        pass
+
+
 # ---------------------------------------------------------------- permute
 def pin_permute_copy():
     rng = np.random.default_rng(51)
@@ -574,7 +632,7 @@ def pin_combine_cases():
 
 PINS = [pin_score_closed_forms, pin_score_library_cases, pin_status_and_nan,
         pin_gate_integer_exact, pin_gate_torch_fp64, pin_hash_lookup, pin_dispatch_library,
-        pin_dispatch_limited, pin_ep_layout, pin_route_grouped,
+        pin_dispatch_limited, pin_ep_layout, pin_route_grouped, pin_expert_ffn,
         pin_permute_copy, pin_combine_cases, pin_weight_invariants, pin_dynamic_k_prefix,
         pin_deepseek_worked_cases, pin_brute_force_selection]
 

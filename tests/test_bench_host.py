@@ -64,3 +64,21 @@ def test_oracle_chain_runs_on_cpu_inputs(bench, name):
     assert bench.oracle_sample_size(wl, inp, 0.05) >= 8
     if wl.k_choices:
         assert set(np.unique(h["kpt"])) <= set(wl.k_choices)
+
+
+def test_oracle_chain_with_experts_on_cpu(bench):
+    from token_dispatch_moe_b200.workloads import make_expert_weights
+    for name in ("mixtral_tiny", "gptoss_top4"):
+        wl = WORKLOADS[name].scaled(200).with_ffn()
+        if name == "gptoss_top4":  # keep the fp64 FFN small on CPU
+            import dataclasses
+            wl = dataclasses.replace(wl, d=64, ffn_dim=32)
+        inp = make_inputs(wl, "cpu", with_y=False)
+        ex = make_expert_weights(wl, "cpu")
+        assert (ex["b1"] is not None) == (wl.ffn_act == "swiglu_oai")
+        h = bench.oracle_inputs(wl, inp, 12, ex)
+        bench.oracle_chain(wl, h)
+        b = bench.stage_bytes(wl, 24, limited=(24, 12, 100))
+        f = bench.stage_flops(wl, 24)
+        assert f["expert_gate_up"] == 2.0 * 24 * 2 * wl.ffn_dim * wl.d
+        assert b["expert_down"] >= wl.E * wl.d * wl.ffn_dim * 2

@@ -57,6 +57,14 @@ MUTANTS = {
     "grouped_candidates_worst": ("cand[nc++] = grp[i];", "cand[nc++] = grp[gsz - 1 - i];"),
     "grouped_no_final_sort": ("        qsort(cand, (size_t)nc, sizeof(ranked), by_key_desc);\n        int32_t *sel = ids + t * k_max;",
                               "        int32_t *sel = ids + t * k_max;"),
+    "oai_no_alpha": ("gc * (1.0 / (1.0 + exp(-ORACLE_OAI_ALPHA * gc))) * (uc + 1.0)",
+                     "gc * (1.0 / (1.0 + exp(-gc))) * (uc + 1.0)"),
+    "oai_no_plus_one": ("exp(-ORACLE_OAI_ALPHA * gc))) * (uc + 1.0)", "exp(-ORACLE_OAI_ALPHA * gc))) * uc"),
+    "swiglu_gate_up_swapped": ("    return g * (1.0 / (1.0 + exp(-g))) * u;", "    return u * (1.0 / (1.0 + exp(-u))) * g;"),
+    "down_transposed": ("const uint16_t *wr = w2 + ((int64_t)e * d + c) * F;",
+                        "const uint16_t *wr = w2 + ((int64_t)e * F + (c % F)) * d;"),
+    "ffn_wrong_expert": ("        if (offsets[e] <= r && r < offsets[e + 1]) return e;",
+                         "        if (offsets[e] <= r && r < offsets[e + 1]) return (e + 1) % E;"),
     "ep_owner_modulo": ("const int32_t d = e / el;", "const int32_t d = e % G;"),
     "ep_sources_reversed": ("if (ids_all[(int64_t)r * n + a] == e) {",
                             "if (ids_all[(int64_t)(G - 1 - r) * n + a] == e) {"),

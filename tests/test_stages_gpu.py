@@ -468,3 +468,65 @@ def test_gate_route_without_logits_and_nan():
         moe.moe_gate_route(x, w, None, None, moe.RouteParams.make(E, 17, "softmax"),
                            torch.empty((T, 17), dtype=torch.int32, device=DEV),
                            torch.empty((T, 17), device=DEV))
+
+
+GROUPED_CASES = [
+    # T, E, G, k_per_group, k, score, renorm, scale, integer logits
+    (1000, 128, 8, 2, 8, "softmax", True, 1.0, False),
+    (777, 256, 8, 4, 8, "sigmoid", True, 2.5, False),
+    (500, 384, 6, 2, 6, "sqrt_softplus", True, 1.0, False),
+    (300, 64, 4, 3, 12, "topk_softmax", True, 1.0, True),   # every candidate kept
+    (257, 512, 32, 1, 32, "sigmoid", False, 1.0, False),
+    (100, 8, 1, 2, 2, "softmax", True, 1.0, False),         # one group: the flat rule
+    (333, 96, 3, 32, 5, "softmax", True, 1.0, True),        # whole groups: the flat rule
+    (200, 30, 3, 2, 4, "softmax", False, 1.0, True),        # E not a multiple of 32
+]
+
+
+@pytest.mark.parametrize("case", GROUPED_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_route_grouped_parity(case):
+    T, E, G, kpg, k, score, renorm, scale, integer = case
+    g = _gen(T + E + kpg)
+    if integer:
+        logits = torch.randint(-3, 4, (T, E), generator=g, device=DEV).float()
+    else:
+        logits = torch.randn((T, E), generator=g, device=DEV)
+    p = moe.RouteParams.make(E, k, score, G, 1, 1, renorm, scale)
+    ids = torch.full((T, k), -7, dtype=torch.int32, device=DEV)
+    w = torch.full((T, k), 7.0, device=DEV)
+    st = _status()
+    moe.moe_route_grouped(logits, p, kpg, ids, w, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    sc = oracle_score(score)
+    o = oracle.route_grouped(logits.cpu().numpy(), k_max=k, score=sc, n_groups=G, k_per_group=kpg,
+                             renormalize=renorm, route_scale=scale, want_keys=True)
+    gi, gw = ids.cpu().numpy(), w.cpu().numpy().astype(np.float64)
+    rows = np.nonzero(~np.all(gi == o["ids"], axis=1))[0]
+    for t in rows:  # only a tie in the oracle's fp64 scores may order them otherwise
+        kg = o["keys"][t][gi[t]]
+        ko = o["keys"][t][o["ids"][t]]
+        assert np.array_equal(np.sort(kg), np.sort(ko)) and np.all(np.isfinite(kg)), \
+            f"row {t}: gpu {gi[t]} oracle {o['ids'][t]}"
+    ow = o["w"].copy()
+    if rows.size:
+        ow[rows] = oracle.weights_for_ids(logits.cpu().numpy()[rows], gi[rows], score=sc,
+                                          renormalize=renorm, route_scale=scale)
+    assert np.all(np.abs(gw - ow) <= 1e-5 * np.abs(ow)), np.max(np.abs(gw - ow) / np.abs(ow))
+    if G == 1 or kpg == E // G:  # the flat router gives the same ids
+        fids = torch.empty_like(ids)
+        fw = torch.empty_like(w)
+        moe.moe_route(logits, None, None, moe.RouteParams.make(E, k, score, 1, 1, 1, renorm, scale),
+                      fids, fw)
+        torch.cuda.synchronize()
+        assert torch.equal(fids, ids)
+
+
+def test_route_grouped_validation():
+    logits = torch.zeros((4, 16), device=DEV)
+    ids = torch.empty((4, 4), dtype=torch.int32, device=DEV)
+    w = torch.empty((4, 4), device=DEV)
+    for E_, G, kpg, k in ((16, 3, 1, 2), (16, 4, 0, 2), (16, 4, 5, 4), (16, 2, 1, 4)):
+        p = moe.RouteParams.make(E_, k, "softmax", G, 1, 1, True, 1.0)
+        with pytest.raises((moe.MoeError, ValueError)):
+            moe.moe_route_grouped(logits, p, kpg, ids[:, :k].contiguous(), w[:, :k].contiguous())

@@ -11,8 +11,8 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_check import (check_combine, check_dispatch, check_dispatch_limited, check_gate,
-                       check_permute, check_route, np32)
+from gpu_check import (check_combine, check_dispatch, check_dispatch_limited, check_expert_h,
+                       check_expert_y, check_gate, check_permute, check_route, np32)
 from token_dispatch_moe_b200.path import RouterDispatch
 from token_dispatch_moe_b200.workloads import WORKLOADS, make_inputs
 
@@ -93,3 +93,34 @@ def test_workload_reduced(name, fused):
 def test_workload_full(name):
     _run_and_check(WORKLOADS[name], sampled=True)
     torch.cuda.empty_cache()
+
+
+FFN_T = {"mixtral_tiny": 253, "qwen3_dynk": 1500, "gptoss_top4": 700}
+
+
+@pytest.mark.parametrize("name", list(FFN_T))
+def test_workload_with_expert_ffn(name):
+    """The chain with the experts' FFN on the permuted rows (expert blocks
+    padded to 128): dispatch bit-exact, h and y against the oracle on sampled
+    token rows (fed the device's previous stage), combine against the oracle
+    over every token."""
+    from token_dispatch_moe_b200 import MOE_ACT_SWIGLU, MOE_ACT_SWIGLU_OAI
+    from token_dispatch_moe_b200.workloads import make_expert_weights
+    wl = WORKLOADS[name].scaled(FFN_T[name]).with_ffn()
+    inp = make_inputs(wl, "cuda", with_y=False)
+    ex = make_expert_weights(wl, "cuda")
+    path = RouterDispatch(wl, keep_logits=True)
+    path.run(inp, experts=ex)
+    torch.cuda.synchronize()
+    assert path.status.item() == 0
+    ids = np32(path.topk_ids)
+    n = check_dispatch_limited(ids, np32(path.counts), np32(path.offsets), np32(path.sorted_token),
+                               np32(path.dest_pos), path.dropped.item(), wl.E, 0, 128)
+    st = np32(path.sorted_token)[:n]
+    real = np.nonzero(st >= 0)[0]
+    rows = np.unique(np.concatenate([_sample(real.size, 96, 5), [0, real.size - 1]]))
+    rows = real[rows]
+    act = MOE_ACT_SWIGLU_OAI if wl.ffn_act == "swiglu_oai" else MOE_ACT_SWIGLU
+    check_expert_h(path.h, path.xs, path.offsets, ex["w1"], ex["w3"], ex["b1"], ex["b3"], act, rows)
+    check_expert_y(path.y, path.h, path.offsets, ex["w2"], ex["b2"], rows)
+    check_combine(path.out, path.y, np32(path.topk_w), np32(path.dest_pos), inp["shared"])

@@ -87,6 +87,9 @@ def load_library(path: str | None = None):
         "moe_dispatch_workspace_size": ([i64, i32, i32, ctypes.POINTER(ctypes.c_size_t)], st),
         "moe_dispatch": ([P, i64, i32, i32, P, P, P, P, P, ctypes.c_size_t, P, P], st),
         "moe_dispatch_static": ([P, i64, i32, i32, P, P, P, P, P, P], st),
+        "moe_expert_gate_up": ([P, P, P, P, P, P, i32, i32, i32, i64, i32, P, P, P], st),
+        "moe_expert_down": ([P, P, P, P, i32, i32, i32, i64, P, P, P], st),
+        "moe_route_grouped": ([P, ctypes.POINTER(RouteParams), i32, i64, P, P, P, P], st),
         "moe_ep_layout": ([P, P, P, P, i32, i32, i64, i32, i32, P, P, P, P, P], st),
         "moe_ep_permute": ([P, P, P, P, i32, i64, i64, i32, i32, P, P], st),
         "moe_ep_combine": ([P, P, P, P, P, i32, i64, i64, i32, i32, P, P, P], st),
@@ -193,6 +196,23 @@ def moe_route(logits, bias, k_per_token, params: RouteParams, topk_ids, topk_w, 
     _check(load_library().moe_route(_ptr(logits), _ptr(bias), _ptr(k_per_token),
                                     ctypes.byref(params), T, _ptr(topk_ids), _ptr(topk_w),
                                     _ptr(d_status), _stream(stream)), "moe_route")
+
+
+def moe_route_grouped(logits, params: RouteParams, k_per_group: int, topk_ids, topk_w,
+                      d_status=None, stream=None):
+    """Per-group candidates (k_per_group best of each contiguous group), then
+    the params.k_max best of them."""
+    _need(logits, torch.float32, "logits", 2)
+    _need(topk_ids, torch.int32, "topk_ids", 2)
+    _need(topk_w, torch.float32, "topk_w", 2)
+    _need(d_status, torch.int32, "d_status")
+    T, E = logits.shape
+    if E != params.num_experts or tuple(topk_ids.shape) != (T, params.k_max) or \
+            tuple(topk_w.shape) != (T, params.k_max):
+        raise ValueError("shape mismatch")
+    _check(load_library().moe_route_grouped(_ptr(logits), ctypes.byref(params), k_per_group, T,
+                                            _ptr(topk_ids), _ptr(topk_w), _ptr(d_status),
+                                            _stream(stream)), "moe_route_grouped")
 
 
 def moe_hash_route(token_ids, tid2eid, logits, params: RouteParams, topk_ids, topk_w,
@@ -328,6 +348,45 @@ def moe_ep_combine(peers_y, dest_rank, dest_row, topk_w, shared, out, recv_capac
                                          _ptr(topk_w), _ptr(shared), peers_y.numel(),
                                          recv_capacity, T, k_max, d, _ptr(out), _ptr(d_status),
                                          _stream(stream)), "moe_ep_combine")
+
+
+MOE_ACT_SWIGLU, MOE_ACT_SWIGLU_OAI = 0, 1
+
+
+def moe_expert_gate_up(xs, offsets, w1, w3, h, b1=None, b3=None, act=MOE_ACT_SWIGLU,
+                       d_status=None, stream=None):
+    """h = act(xs W1[e]^T + b1[e], xs W3[e]^T + b3[e]) per 128-row-aligned expert block."""
+    for t, n in ((xs, "xs"), (w1, "w1"), (w3, "w3"), (h, "h")):
+        _need(t, torch.bfloat16, n)
+    _need(offsets, torch.int32, "offsets", 1)
+    _need(b1, torch.float32, "b1")
+    _need(b3, torch.float32, "b3")
+    _need(d_status, torch.int32, "d_status")
+    E, F, d = w1.shape
+    rows = xs.shape[0]
+    if tuple(w3.shape) != (E, F, d) or xs.shape[1] != d or tuple(h.shape) != (rows, F) or \
+            offsets.numel() != E + 1:
+        raise ValueError("shape mismatch")
+    _check(load_library().moe_expert_gate_up(_ptr(xs), _ptr(offsets), _ptr(w1), _ptr(w3), _ptr(b1),
+                                             _ptr(b3), E, d, F, rows, act, _ptr(h),
+                                             _ptr(d_status), _stream(stream)),
+           "moe_expert_gate_up")
+
+
+def moe_expert_down(h, offsets, w2, y, b2=None, d_status=None, stream=None):
+    """y = h W2[e]^T + b2[e] per 128-row-aligned expert block."""
+    for t, n in ((h, "h"), (w2, "w2"), (y, "y")):
+        _need(t, torch.bfloat16, n)
+    _need(offsets, torch.int32, "offsets", 1)
+    _need(b2, torch.float32, "b2")
+    _need(d_status, torch.int32, "d_status")
+    E, d, F = w2.shape
+    rows = h.shape[0]
+    if h.shape[1] != F or tuple(y.shape) != (rows, d) or offsets.numel() != E + 1:
+        raise ValueError("shape mismatch")
+    _check(load_library().moe_expert_down(_ptr(h), _ptr(offsets), _ptr(w2), _ptr(b2), E, d, F,
+                                          rows, _ptr(y), _ptr(d_status), _stream(stream)),
+           "moe_expert_down")
 
 
 def moe_dispatch_static(topk_ids, E, counts, offsets, sorted_token, dest_pos, d_status=None,

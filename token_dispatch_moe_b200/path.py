@@ -9,9 +9,10 @@ from __future__ import annotations
 
 import torch
 
-from . import (RouteParams, moe_combine, moe_dispatch, moe_dispatch_limited,
-               moe_dispatch_limited_rows, moe_dispatch_workspace_size, moe_gate_gemm,
-               moe_gate_route, moe_hash_route, moe_permute, moe_route)
+from . import (MOE_ACT_SWIGLU, MOE_ACT_SWIGLU_OAI, RouteParams, moe_combine, moe_dispatch,
+               moe_dispatch_limited, moe_dispatch_limited_rows, moe_dispatch_workspace_size,
+               moe_expert_down, moe_expert_gate_up, moe_gate_gemm, moe_gate_route,
+               moe_hash_route, moe_permute, moe_route)
 from .workloads import Workload
 
 
@@ -59,6 +60,12 @@ class RouterDispatch:
         self.out = (torch.empty((T, wl.d), dtype=torch.bfloat16, device=device)
                     if wl.combine else None)
         self.status = torch.zeros((1,), **i32)
+        self.h = self.y = None
+        if wl.ffn_dim and wl.pad % 128 == 0:  # the experts' FFN can run on these blocks
+            self.h = torch.empty((max(self.expert_rows, 1), wl.ffn_dim), dtype=torch.bfloat16,
+                                 device=device)
+            self.y = torch.empty((max(self.expert_rows, 1), wl.d), dtype=torch.bfloat16,
+                                 device=device)
         if wl.hash_vocab:
             self.hash_ids = torch.empty((T, k), **i32)
             self.hash_w = torch.empty((T, k), dtype=torch.float32, device=device)
@@ -96,11 +103,21 @@ class RouterDispatch:
     def combine(self, y, shared=None, stream=None):
         moe_combine(y, self.topk_w, self.dest_pos, shared, self.out, stream)
 
+    def expert_gate_up(self, weights: dict, stream=None):
+        act = MOE_ACT_SWIGLU_OAI if self.wl.ffn_act == "swiglu_oai" else MOE_ACT_SWIGLU
+        moe_expert_gate_up(self.xs, self.offsets, weights["w1"], weights["w3"], self.h,
+                           weights["b1"], weights["b3"], act, self.status, stream)
+
+    def expert_down(self, weights: dict, stream=None):
+        moe_expert_down(self.h, self.offsets, weights["w2"], self.y, weights["b2"], self.status,
+                        stream)
+
     # The whole chain -----------------------------------------------------------
-    def run(self, inputs: dict, stream=None):
+    def run(self, inputs: dict, stream=None, experts: dict | None = None):
         """gate (if the workload has one) -> route -> dispatch -> permute ->
-        combine (if the workload ends there).  ``inputs`` as made by
-        :func:`workloads.make_inputs`."""
+        [experts' FFN, when ``experts`` holds their weights] -> combine (if the
+        workload ends there).  ``inputs`` as made by :func:`workloads.make_inputs`;
+        without experts the combine reads the synthetic ``inputs["y"]``."""
         if self.fused:
             self.gate_route(inputs["x"], inputs["w"], inputs["bias"], inputs["k_per_token"], stream)
         else:
@@ -109,8 +126,13 @@ class RouterDispatch:
             self.route(logits, inputs["bias"], inputs["k_per_token"], stream)
         self.dispatch(stream=stream)
         self.permute(inputs["x"], stream)
+        y = inputs["y"]
+        if experts is not None:
+            self.expert_gate_up(experts, stream)
+            self.expert_down(experts, stream)
+            y = self.y
         if self.wl.combine:
-            self.combine(inputs["y"], inputs["shared"], stream)
+            self.combine(y, inputs["shared"], stream)
         return self.out if self.wl.combine else self.xs
 
     def run_hash_layer(self, inputs: dict, logits=None, stream=None):

@@ -19,6 +19,9 @@ gives the expert counts, k, scoring and shared experts of the families;
                  one shared expert; logits ~N(0,1), 10% of rows +3 on 4 hot experts
   gptoss_top4    T=262144, d=2880, E=128, k=4, gpt-oss (softmax over the 4
                  selected logits); logits as llama4_top1
+  with_ffn()      mixtral_tiny, qwen3_dynk and gptoss_top4 also run their experts'
+                 SwiGLU FFN (F = 256, 768, 2880; gpt-oss: clamped SwiGLU with
+                 biases) on the permuted rows, with synthetic weights
   llama4_top1_capacity
                  llama4_top1 with a Switch-style capacity (factor 1.0: each
                  expert keeps at most T/E = 2048 tokens, the skewed hot experts
@@ -59,6 +62,8 @@ class Workload:
     w_std: float = 0.02
     capacity_factor: float = 0.0   # > 0: per-expert capacity ceil(cf * T * k / E)
     pad: int = 1                   # expert blocks padded to a multiple of this many rows
+    ffn_dim: int = 0               # expert FFN width F (0: no FFN model for this family)
+    ffn_act: str = "swiglu"        # "swiglu" or "swiglu_oai" (gpt-oss, with biases)
 
     @property
     def limited(self) -> bool:
@@ -75,12 +80,20 @@ class Workload:
         """Same workload with another token count (smaller parity cases)."""
         return dataclasses.replace(self, T=T)
 
+    def with_ffn(self) -> "Workload":
+        """The workload with its experts' FFN run on the permuted rows: expert
+        blocks padded to the 128-row tiles of the grouped GEMMs."""
+        if not self.ffn_dim:
+            raise ValueError(f"{self.name} has no expert FFN shape")
+        return dataclasses.replace(self, pad=max(self.pad, 128))
+
 
 WORKLOADS = {
     w.name: w for w in [
-        Workload("mixtral_tiny", 1, T=256, d=128, E=8, k_max=2, score="softmax", gate=False),
+        Workload("mixtral_tiny", 1, T=256, d=128, E=8, k_max=2, score="softmax", gate=False,
+                 ffn_dim=256),
         Workload("qwen3_dynk", 2, T=16384, d=2048, E=128, k_max=16, score="softmax", gate=True,
-                 k_choices=(4, 8, 16)),
+                 k_choices=(4, 8, 16), ffn_dim=768),
         Workload("deepseek_v3", 3, T=65536, d=7168, E=256, k_max=8, score="sigmoid", gate=True,
                  bias=True, n_groups=8, topk_groups=4, group_topn=2, route_scale=2.5,
                  shared=True),
@@ -89,7 +102,7 @@ WORKLOADS = {
         Workload("llama4_top1", 5, T=262144, d=5120, E=128, k_max=1, score="sigmoid",
                  gate=False, renormalize=False, shared=True, skew=True),
         Workload("gptoss_top4", 6, T=262144, d=2880, E=128, k_max=4, score="topk_softmax",
-                 gate=False, skew=True),
+                 gate=False, skew=True, ffn_dim=2880, ffn_act="swiglu_oai"),
         Workload("llama4_top1_capacity", 7, T=262144, d=5120, E=128, k_max=1, score="sigmoid",
                  gate=False, renormalize=False, shared=True, skew=True, capacity_factor=1.0,
                  pad=128),
@@ -108,6 +121,22 @@ def normal_bf16(shape, std, device, seed):
     if std != 1.0:
         t.mul_(std)
     return t.to(torch.bfloat16)
+
+
+def make_expert_weights(wl: Workload, device="cuda", seed_offset: int = 0) -> dict:
+    """Synthetic expert FFN weights: W1, W3 [E][F][d] ~N(0, 1/d), W2 [E][d][F]
+    ~N(0, 1/F) in bf16 (so the projections are O(1) for O(1) inputs); for the
+    gpt-oss activation also biases b1, b3 [E][F] and b2 [E][d] ~N(0, 0.5^2)."""
+    s = 1000 * wl.index + 20 + seed_offset
+    E, d, F = wl.E, wl.d, wl.ffn_dim
+    out = {"w1": normal_bf16((E, F, d), d ** -0.5, device, s),
+           "w3": normal_bf16((E, F, d), d ** -0.5, device, s + 1),
+           "w2": normal_bf16((E, d, F), F ** -0.5, device, s + 2),
+           "b1": None, "b3": None, "b2": None}
+    if wl.ffn_act == "swiglu_oai":
+        for i, (name, shape) in enumerate((("b1", (E, F)), ("b3", (E, F)), ("b2", (E, d)))):
+            out[name] = torch.randn(shape, generator=_gen(device, s + 3 + i), device=device) * 0.5
+    return out
 
 
 def k_per_token(wl: Workload, device, seed=None):
