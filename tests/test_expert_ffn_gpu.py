@@ -66,6 +66,7 @@ FFN_CASES = [
     (300, 8, 4, 2048, 768, moe.MOE_ACT_SWIGLU, False, False),      # the qwen3 expert shape
     (200, 4, 4, 2880, 2880, moe.MOE_ACT_SWIGLU_OAI, True, False),  # the gpt-oss expert shape
     (129, 1, 3, 64, 32, moe.MOE_ACT_SWIGLU, True, True),
+    (4000, 8, 8, 512, 256, moe.MOE_ACT_SWIGLU, False, True),      # several tiles per CTA
 ]
 
 

@@ -14,15 +14,18 @@
 //   swiglu_oai: g' = min(g, limit), u' = clamp(u, -limit, limit),
 //               act = g' * sigmoid(alpha * g') * (u' + 1)
 //
-// sm_100a design: one 128-row M tile of one expert per CTA (expert blocks are
-// 128-row aligned, so a tile never straddles two experts) and one N tile of
-// BN output columns; grid (N tiles, M tiles), N fastest so CTAs that share an
-// A tile run together and find it in L2.  Warp 0 issues TMA loads (A tile and,
-// for gate_up, the W1 and W3 tiles of the same columns), one thread of warp 1
-// issues tcgen05.mma into TMEM (gate_up: two accumulators side by side), warp
-// 2 owns the TMEM columns, warps 4..7 run the epilogue (tcgen05.ld, bias,
-// activation, bf16 stores of the CTA's rows).  Tiles past the last expert
-// block exit at once.  Every mbarrier wait is bounded.
+// sm_100a design: a persistent grid, one CTA per SM, walks output tiles of
+// 128 rows of one expert (expert blocks are 128-row aligned, so a tile never
+// straddles two experts) by BN columns, N tile fastest so the CTAs running
+// together share their A tile in L2.  Warp 0 issues TMA loads (the A tile and,
+// for gate_up, the W1 and W3 tiles of the same columns) into a stage ring that
+// runs on across tiles; one thread of warp 1 issues tcgen05.mma into one of
+// two TMEM accumulators (gate_up: gate and up side by side in each); warp 2
+// owns the TMEM columns; warps 4..7 run the epilogue (tcgen05.ld, bias,
+// activation, bf16 stores of the tile's rows) of tile j while the MMAs of tile
+// j+1 fill the other accumulator.  Every mbarrier wait is bounded; a wait that
+// gives up stops every role, and the CTA drains its copies and MMAs before it
+// frees the TMEM.
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -65,62 +68,72 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// The expert whose 128-row-aligned block holds the M tile starting at row m0
+// (off = the offsets, staged in shared memory), or -1 when the tile lies past
+// the last block or straddles two blocks (offsets not 128-aligned).  Every
+// role of the CTA walks the same tiles through this function.
+__device__ __forceinline__ int tile_expert(const int32_t *off, int E, int64_t total, int64_t m0) {
+    if (m0 >= total) return -1;
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {  // the last e with off[e] <= m0 (offsets ascend)
+        const int mid = (lo + hi + 1) >> 1;
+        if ((int64_t)off[mid] <= m0) lo = mid; else hi = mid - 1;
+    }
+    if ((off[lo] & (kFBM - 1)) != 0 || m0 + kFBM > (int64_t)off[lo + 1]) return -1;
+    return lo;
+}
+
 // GATE_UP: A = xs, B0 = W1, B1 = W3, out = h.  Otherwise A = h, B0 = W2, out = y.
+// Persistent: one CTA per SM walks tiles blockIdx.x, +gridDim.x, ...; the
+// shared-memory stage ring runs on across tiles, and two TMEM accumulators
+// alternate so the epilogue of one tile overlaps the mainloop of the next.
 template <bool GATE_UP>
 __global__ void __launch_bounds__(kFThreads, 1)
     expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                        const __grid_constant__ CUtensorMap tmap_b0,
                        const __grid_constant__ CUtensorMap tmap_b1, const FfnArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    __shared__ int expert_s;
+    __shared__ int abort_s;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * a.BN;
-    const int64_t m0 = (int64_t)blockIdx.y * kFBM;
-
-    // Which expert block holds this tile (last e with offsets[e] <= m0).
-    if (threadIdx.x == 0) {
-        int e = -1;
-        const int64_t total = a.offsets[a.E];
-        if (m0 < total && total <= a.rows) {
-            int lo = 0, hi = a.E - 1;
-            while (lo < hi) {  // offsets ascend; find the last e with offsets[e] <= m0
-                const int mid = (lo + hi + 1) >> 1;
-                if ((int64_t)a.offsets[mid] <= m0) lo = mid; else hi = mid - 1;
-            }
-            e = lo;
-            if ((a.offsets[e] & (kFBM - 1)) != 0 || m0 + kFBM > (int64_t)a.offsets[e + 1]) {
-                report(a.status, MOE_ERR_DEVICE_INDEX);  // blocks not 128-row aligned
-                e = -1;
-            }
-        } else if (total > a.rows) {
-            report(a.status, MOE_ERR_DEVICE_INDEX);
-        }
-        expert_s = e;
-    }
-    __syncthreads();
-    const int e = expert_s;
-    if (e < 0) return;  // past the last block (or bad offsets): nothing to do
+    const int n_tiles = a.N / a.BN;
+    const int64_t total = __ldg(a.offsets + a.E);
+    const int64_t m_tiles = total > 0 && total <= a.rows ? (total + kFBM - 1) / kFBM : 0;
+    const int64_t num_tiles = m_tiles * n_tiles;
+    if (threadIdx.x == 0 && blockIdx.x == 0 && total > a.rows)
+        report(a.status, MOE_ERR_DEVICE_INDEX);  // blocks reach past the buffers: no tile runs
+    if ((int64_t)blockIdx.x >= num_tiles) return;  // nothing for this CTA
 
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *const gbase = smem_raw + (base - raw);
     const int S = a.stages;
+    // [stages][full[S]][empty[S]][tmem_full[2]][tmem_empty[2]][drain][tmem slot]
     const uint32_t bar0 = base + (uint32_t)S * a.stage_bytes;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
-    const uint32_t tmem_full_bar = bar0 + 8u * (2 * S);
+    auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * S + b); };
+    auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * S + 2 + b); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * S + 4);
     uint32_t *tmem_slot =
-        reinterpret_cast<uint32_t *>(gbase + (size_t)S * a.stage_bytes + 8u * (2 * S + 1));
+        reinterpret_cast<uint32_t *>(gbase + (size_t)S * a.stage_bytes + 8u * (2 * S + 5));
+    int32_t *off = reinterpret_cast<int32_t *>(gbase + (size_t)S * a.stage_bytes + 256);
     const uint32_t btile = (uint32_t)a.BN * 128u;  // bytes of one BN x 64 operand tile
+    const uint32_t acc_cols = GATE_UP ? 2u * a.BN : (uint32_t)a.BN;
 
     if (threadIdx.x == 0) {
+        abort_s = 0;
         for (int s = 0; s < S; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
-        mbar_init(tmem_full_bar, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull_bar(b), 1);
+            mbar_init(tempty_bar(b), 4);  // one arrival per epilogue warp
+        }
+        mbar_init(drain_bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    for (int i = threadIdx.x; i <= a.E; i += blockDim.x) off[i] = __ldg(a.offsets + i);
     if (warp == 2) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(tmem_slot)),
@@ -132,50 +145,99 @@ __global__ void __launch_bounds__(kFThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int brow = e * a.N + n0;  // first weight row of this tile in the [E*N][K] view
+    volatile int *abort_v = &abort_s;
 
     if (warp == 0 && lane == 0) {
-        int issued = 0;
-        for (int kb = 0; kb < a.num_kb; ++kb) {
-            const int s = kb % S;
-            const uint32_t ph = (uint32_t)(kb / S) & 1u;
-            if (!mbar_wait(empty_bar(s), ph ^ 1u, a.status)) break;
-            const uint32_t st = base + (uint32_t)s * a.stage_bytes;
-            mbar_arrive_expect_tx(full_bar(s), a.stage_bytes);
-            tma_load_2d(st, &tmap_a, full_bar(s), kb * kFBK, (int)m0);
-            tma_load_2d(st + kFATile, &tmap_b0, full_bar(s), kb * kFBK, brow);
-            if (GATE_UP) tma_load_2d(st + kFATile + btile, &tmap_b1, full_bar(s), kb * kFBK, brow);
-            issued = kb + 1;
-        }
-        for (int kb = issued - S < 0 ? 0 : issued - S; kb < issued; ++kb)
-            if (!mbar_wait(full_bar(kb % S), (uint32_t)(kb / S) & 1u, a.status)) break;
-    } else if (warp == 1 && lane == 0) {
-        for (int kb = 0; kb < a.num_kb; ++kb) {
-            const int s = kb % S;
-            const uint32_t ph = (uint32_t)(kb / S) & 1u;
-            if (!mbar_wait(full_bar(s), ph, a.status)) break;
-            tc_fence_after();
-            const uint32_t st = base + (uint32_t)s * a.stage_bytes;
-#pragma unroll
-            for (int k = 0; k < kFBK / kFUmmaK; ++k) {
-                const uint32_t koff = (uint32_t)(k * kFUmmaK * 2);
-                const uint64_t adesc = sw128_desc(st + koff);
-                const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-                umma_bf16(tmem_base, adesc, sw128_desc(st + kFATile + koff), a.idesc, acc);
+        // TMA producer: the stage ring runs on across tiles.
+        uint32_t it = 0;
+        for (int64_t t = blockIdx.x; t < num_tiles && !*abort_v; t += gridDim.x) {
+            const int64_t m0 = (t / n_tiles) * kFBM;
+            const int e = tile_expert(off, a.E, total, m0);
+            if (e < 0) continue;
+            const int brow = e * a.N + (int)(t % n_tiles) * a.BN;
+            for (int kb = 0; kb < a.num_kb; ++kb, ++it) {
+                const int s = (int)(it % (uint32_t)S);
+                const uint32_t ph = (it / (uint32_t)S) & 1u;
+                if (!mbar_wait(empty_bar(s), ph ^ 1u, a.status)) {
+                    *abort_v = 1;
+                    break;
+                }
+                const uint32_t st = base + (uint32_t)s * a.stage_bytes;
+                mbar_arrive_expect_tx(full_bar(s), a.stage_bytes);
+                tma_load_2d(st, &tmap_a, full_bar(s), kb * kFBK, (int)m0);
+                tma_load_2d(st + kFATile, &tmap_b0, full_bar(s), kb * kFBK, brow);
                 if (GATE_UP)
-                    umma_bf16(tmem_base + (uint32_t)a.BN, adesc,
-                              sw128_desc(st + kFATile + btile + koff), a.idesc, acc);
+                    tma_load_2d(st + kFATile + btile, &tmap_b1, full_bar(s), kb * kFBK, brow);
             }
-            umma_commit(empty_bar(s));
         }
-        umma_commit(tmem_full_bar);
+        // Drain: the last load into every stage has landed before the CTA exits.
+        const uint32_t first = it > (uint32_t)S ? it - (uint32_t)S : 0u;
+        for (uint32_t i = first; i < it; ++i)
+            if (!mbar_wait(full_bar((int)(i % (uint32_t)S)), (i / (uint32_t)S) & 1u, a.status))
+                break;
+    } else if (warp == 1 && lane == 0) {
+        // MMA issuer: accumulator b = j & 1 of the j-th tile this CTA computes.
+        uint32_t it = 0, j = 0;
+        for (int64_t t = blockIdx.x; t < num_tiles && !*abort_v; t += gridDim.x) {
+            if (tile_expert(off, a.E, total, (t / n_tiles) * kFBM) < 0) continue;
+            const uint32_t b = j & 1u;
+            if (!mbar_wait(tempty_bar((int)b), ((j >> 1) & 1u) ^ 1u, a.status)) {
+                *abort_v = 1;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t acc = tmem_base + b * acc_cols;
+            for (int kb = 0; kb < a.num_kb; ++kb, ++it) {
+                const int s = (int)(it % (uint32_t)S);
+                const uint32_t ph = (it / (uint32_t)S) & 1u;
+                if (!mbar_wait(full_bar(s), ph, a.status)) {
+                    *abort_v = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t st = base + (uint32_t)s * a.stage_bytes;
+#pragma unroll
+                for (int k = 0; k < kFBK / kFUmmaK; ++k) {
+                    const uint32_t koff = (uint32_t)(k * kFUmmaK * 2);
+                    const uint64_t adesc = sw128_desc(st + koff);
+                    const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
+                    umma_bf16(acc, adesc, sw128_desc(st + kFATile + koff), a.idesc, accum);
+                    if (GATE_UP)
+                        umma_bf16(acc + (uint32_t)a.BN, adesc,
+                                  sw128_desc(st + kFATile + btile + koff), a.idesc, accum);
+                }
+                umma_commit(empty_bar(s));
+            }
+            if (*abort_v) break;
+            umma_commit(tfull_bar((int)b));
+            ++j;
+        }
+        // Every MMA issued above has completed before the columns are freed.
+        umma_commit(drain_bar);
+        mbar_wait(drain_bar, 0u, a.status);
     } else if (warp >= 4) {
+        // Epilogue: warp w reads TMEM lanes 32*(w%4).. = rows of the tile.
         const int q = warp & 3;
-        const bool ok = __all_sync(MOE_FULL_MASK, mbar_wait(tmem_full_bar, 0u, a.status));
-        tc_fence_after();
-        const int64_t row = m0 + q * 32 + lane;
-        const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16);
-        if (ok) {
+        uint32_t j = 0;
+        for (int64_t t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+            const int64_t m0 = (t / n_tiles) * kFBM;
+            const int e = tile_expert(off, a.E, total, m0);
+            if (e < 0) {  // a tile straddling two blocks: skipped by every role, reported here
+                if (q == 0 && lane == 0) report(a.status, MOE_ERR_DEVICE_INDEX);
+                continue;
+            }
+            const uint32_t b = j & 1u;
+            const bool ok = __all_sync(MOE_FULL_MASK,
+                                       !*abort_v && mbar_wait(tfull_bar((int)b), (j >> 1) & 1u,
+                                                              a.status));
+            if (!ok) {
+                if (lane == 0) *abort_v = 1;
+                break;
+            }
+            tc_fence_after();
+            const int n0 = (int)(t % n_tiles) * a.BN;
+            const int64_t row = m0 + q * 32 + lane;
+            const uint32_t trow = tmem_base + b * acc_cols + ((uint32_t)(q * 32) << 16);
             const float *b0 = a.bias0 ? a.bias0 + (int64_t)e * a.N + n0 : nullptr;
             const float *b1 = a.bias1 ? a.bias1 + (int64_t)e * a.N + n0 : nullptr;
             moe_bf16_t *dst = a.out + row * a.N + n0;
@@ -205,6 +267,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
                                        pack2(v[12], v[13]), pack2(v[14], v[15]));
                 }
             }
+            // This warp's reads of accumulator b are done: the MMA may reuse it.
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty_bar((int)b));
+            ++j;
         }
     }
 
@@ -235,9 +302,10 @@ moe_status launch_expert_gemm(const moe_bf16_t *A, const moe_bf16_t *B0, const m
     a.BN = pick_bn(a.N, GATE_UP);
     if (a.BN == 0) return MOE_ERR_UNSUPPORTED;
     a.num_kb = (K + kFBK - 1) / kFBK;
-    const int ncols = GATE_UP ? 2 * a.BN : a.BN;
+    const int ncols = 2 * (GATE_UP ? 2 * a.BN : a.BN);  // two accumulators
     int cols = 32;
     while (cols < ncols) cols *= 2;
+    if (cols > 512) return MOE_ERR_UNSUPPORTED;
     a.tmem_cols = cols;
     a.stage_bytes = (uint32_t)(kFATile + (GATE_UP ? 2 : 1) * a.BN * 128);
     a.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(a.BN >> 3) << 17) |
@@ -249,8 +317,9 @@ moe_status launch_expert_gemm(const moe_bf16_t *A, const moe_bf16_t *B0, const m
         cudaGetLastError();
         return MOE_ERR_CUDA;
     }
-    const int overhead = 1024 + 256;
-    int stages = (int)((max_smem - overhead) / (int)a.stage_bytes);
+    // alignment slack, barriers and TMEM slot, the staged offsets
+    const int overhead = 1024 + 256 + ((a.E + 1) * 4 + 15) / 16 * 16;
+    int stages = (int)((max_smem - 1024 - overhead) / (int)a.stage_bytes);  // 1 KB static
     if (stages > 6) stages = 6;
     if (stages < 2) return MOE_ERR_UNSUPPORTED;
     a.stages = stages;
@@ -265,8 +334,11 @@ moe_status launch_expert_gemm(const moe_bf16_t *A, const moe_bf16_t *B0, const m
         cudaGetLastError();
         return MOE_ERR_CUDA;
     }
-    const dim3 grid((unsigned)(a.N / a.BN), (unsigned)((rows + kFBM - 1) / kFBM));
-    expert_gemm_kernel<GATE_UP><<<grid, kFThreads, smem, as_cuda(stream)>>>(ma, mb0, mb1, a);
+    // Persistent: one CTA per SM, never more CTAs than the largest tile count.
+    const int64_t most = (int64_t)(a.N / a.BN) * ((rows + kFBM - 1) / kFBM);
+    const int64_t grid = most < (int64_t)sm_count() ? most : (int64_t)sm_count();
+    expert_gemm_kernel<GATE_UP><<<(unsigned)grid, kFThreads, smem, as_cuda(stream)>>>(ma, mb0,
+                                                                                      mb1, a);
     return launch_status();
 }
 
@@ -276,7 +348,7 @@ moe_status check_ffn(const void *A, const int32_t *offsets, int32_t E, int32_t d
         return MOE_ERR_INVALID_ARG;
     if (rows == 0) return MOE_OK;
     if (!A || !offsets || !out || !aligned16(A) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
-    if ((rows + kFBM - 1) / kFBM > 65535 || (int64_t)E * (d > F ? d : F) >= (int64_t)INT32_MAX)
+    if (rows >= (int64_t)INT32_MAX || (int64_t)E * (d > F ? d : F) >= (int64_t)INT32_MAX)
         return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
 }
