@@ -90,6 +90,19 @@ def rank_seed_offset(rank: int) -> int:
 
 
 # ------------------------------------------------------------------ byte model
+def hash_stage_bytes(wl) -> dict:
+    """The hash-routed layer's chain: gate GEMM (its logits give the weights),
+    hash_route, dispatch, permute (every token takes k = k_max slots)."""
+    T, d, E, k = wl.T, wl.d, wl.E, wl.k_max
+    n = T * k
+    return {"gate_gemm": T * d * 2 + E * d * 2 + T * E * 4,
+            # token ids, the looked-up table rows, the logits of the k looked-up
+            # experts, ids and weights out
+            "hash_route": T * 4 + n * 4 + n * 4 + n * 8,
+            "dispatch": n * 4 + n * 4 + n * 4 + 8 * E,
+            "permute": T * d * 2 + n * d * 2 + n * 4}
+
+
 def stage_bytes(wl, n_assign: int, fused: bool = False, limited=None) -> dict:
     """Algorithmic DRAM bytes per launch of each kernel (each read once, each
     write once) and the gate's FLOPs.  limited = (kept slots, tokens with a
@@ -240,6 +253,9 @@ def oracle_inputs(wl, inp: dict, n_tokens: int, experts=None) -> dict:
     n += wl.E * (wl.pad - 1)  # padded expert blocks
     h["y"] = bits(normal_bf16((max(n, 1), wl.d), 1.0, "cpu", 1000 * wl.index + 44))
     h["shared"] = bits(inp["shared"][:n_tokens]) if inp["shared"] is not None else None
+    h["token_ids"] = (inp["token_ids"][:n_tokens].cpu().numpy()
+                      if inp.get("token_ids") is not None else None)
+    h["tid2eid"] = inp["tid2eid"].cpu().numpy() if inp.get("tid2eid") is not None else None
     h["experts"] = None
     if experts is not None:
         h["experts"] = {k: (None if v is None else
@@ -248,14 +264,22 @@ def oracle_inputs(wl, inp: dict, n_tokens: int, experts=None) -> dict:
     return h
 
 
-def oracle_chain(wl, h: dict) -> None:
+def oracle_chain(wl, h: dict, hash_layer: bool = False) -> None:
     """The path computed by the fp64 CPU oracle (single thread): gate, route,
     dispatch, permute, [the experts' FFN when h holds their weights], combine,
-    on the sample held in h."""
+    on the sample held in h; or the hash-routed layer's chain (gate, hash
+    route, dispatch, permute)."""
     import oracle
     score = {"softmax": oracle.SOFTMAX, "sigmoid": oracle.SIGMOID,
              "sqrt_softplus": oracle.SQRT_SOFTPLUS, "topk_softmax": oracle.TOPK_SOFTMAX}[wl.score]
     logits = oracle.gate_rows(h["x"], h["w"]).astype(np.float32) if wl.gate else h["logits"]
+    if hash_layer:
+        r = oracle.hash_route(h["token_ids"], h["tid2eid"], num_experts=wl.E, logits=logits,
+                              score=score, renormalize=wl.renormalize,
+                              route_scale=wl.route_scale)
+        dsp = oracle.dispatch(r["ids"], wl.E)
+        oracle.permute(h["x"], dsp["dest_pos"], int(dsp["offsets"][-1]))
+        return
     r = oracle.route(logits, k_max=wl.k_max, score=score, bias=h["bias"], k_per_token=h["kpt"],
                      n_groups=wl.n_groups, topk_groups=wl.topk_groups, group_topn=wl.group_topn,
                      renormalize=wl.renormalize, route_scale=wl.route_scale)
@@ -283,12 +307,12 @@ def oracle_chain(wl, h: dict) -> None:
                        h["shared"], want_mag=False)
 
 
-def oracle_sample_size(wl, inp, budget_s: float, experts=None) -> int:
+def oracle_sample_size(wl, inp, budget_s: float, experts=None, hash_layer=False) -> int:
     """Tokens of CPU work that take about budget_s seconds (calibrated on a small run)."""
     n0 = min(64 if experts is None else 8, wl.T)
     h = oracle_inputs(wl, inp, n0, experts)
     t0 = time.perf_counter()
-    oracle_chain(wl, h)
+    oracle_chain(wl, h, hash_layer)
     per_token = (time.perf_counter() - t0) / n0
     return int(max(8, min(wl.T, budget_s / max(per_token, 1e-9))))
 
@@ -320,11 +344,17 @@ def run_ours(args):
         experts = make_expert_weights(wl, device, seed_offset=rank_seed_offset(rank))
     inp = make_inputs(wl, device, with_y=experts is None, seed_offset=rank_seed_offset(rank))
     n_assign = num_assignments(wl, inp["k_per_token"])
-    path = RouterDispatch(wl, device, fused=False if args.separate else (True if args.fused else None))
+    if args.hash_layer:
+        if not wl.hash_vocab or experts is not None:
+            raise SystemExit("--hash-layer needs a workload with a hash-routed layer, without --ffn")
+        path = RouterDispatch(wl, device, fused=False, keep_logits=True)
+    else:
+        path = RouterDispatch(wl, device,
+                              fused=False if args.separate else (True if args.fused else None))
     stream = torch.cuda.current_stream(device)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=device)
-    bytes_per = stage_bytes(wl, n_assign, path.fused)
+    bytes_per = hash_stage_bytes(wl) if args.hash_layer else stage_bytes(wl, n_assign, path.fused)
     names = list(bytes_per)
 
     def run_step(mark):
@@ -338,6 +368,16 @@ def run_ours(args):
             i += 1
 
         boundary()
+        if args.hash_layer:
+            logits = path.gate(inp["x"], inp["w"])
+            boundary()
+            path.hash_route(inp["token_ids"], inp["tid2eid"], logits)
+            boundary()
+            path.dispatch(path.hash_ids)
+            boundary()
+            path.permute(inp["x"])
+            boundary()
+            return
         if path.fused:
             path.gate_route(inp["x"], inp["w"], inp["bias"], inp["k_per_token"])
             boundary()
@@ -469,7 +509,8 @@ def run_ours(args):
 
     e2e = None
     if not args.no_e2e:
-        e2e = measure_e2e(wl, inp, path, device, stream, min(K, args.e2e_steps), world, experts)
+        e2e = measure_e2e(wl, inp, path, device, stream, min(K, args.e2e_steps), world, experts,
+                          args.hash_layer)
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -477,6 +518,7 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
         "data": "synthetic",
         "config": {"workload": (wl.name + ("+ffn" if experts is not None else "")
+                                + ("/hash-layer" if args.hash_layer else "")
                                 + (f"@T={wl.T}" if args.tokens else "")),
                    "tokens_per_gpu": wl.T, "hidden": wl.d, "experts": wl.E,
                    "k": (f"{'/'.join(map(str, wl.k_choices))} per {wl.segment}-token request"
@@ -491,27 +533,29 @@ def run_ours(args):
                        "pad_rows_to": wl.pad, "kept_slots": limited[0],
                        "dropped_slots": n_assign - limited[0]} if limited else {})},
         "roofline": roofline, "stages": stages, "clocks": clk.summary(),
-        "gpu_launches": (chain_launches(wl, path.fused) + (2 if experts is not None else 0)) * K,
+        "gpu_launches": (5 if args.hash_layer else
+                         chain_launches(wl, path.fused) + (2 if experts is not None else 0)) * K,
         "e2e": e2e,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(wl, inp, args.cpu_budget, experts)
+        result["cpu_baseline"] = cpu_baseline(wl, inp, args.cpu_budget, experts, args.hash_layer)
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
 
 
-def measure_e2e(wl, inp, path, device, stream, steps, world, experts=None):
+def measure_e2e(wl, inp, path, device, stream, steps, world, experts=None, hash_layer=False):
     """Same metric through the C ABI with host buffers: each step copies its
     inputs from pinned host memory, runs the chain and copies the result back."""
-    names = [k for k in ("x", "w", "logits", "bias", "k_per_token", "y", "shared") if
-             inp[k] is not None]
+    keys = ("x", "w", "token_ids") if hash_layer else \
+        ("x", "w", "logits", "bias", "k_per_token", "y", "shared")
+    names = [k for k in keys if inp[k] is not None]
     host = {k: inp[k].cpu().pin_memory() for k in names}
     dev = {k: torch.empty_like(inp[k]) for k in names}
     full = dict(inp)
     full.update(dev)
-    result_dev = path.out if wl.combine else path.xs
+    result_dev = path.out if (wl.combine and not hash_layer) else path.xs
     out_host = torch.empty(result_dev.shape, dtype=result_dev.dtype, pin_memory=True)
     h2d = sum(host[k].numel() * host[k].element_size() for k in names)
     d2h = out_host.numel() * out_host.element_size()
@@ -519,7 +563,10 @@ def measure_e2e(wl, inp, path, device, stream, steps, world, experts=None):
     def one():
         for k in names:
             dev[k].copy_(host[k], non_blocking=True)
-        path.run(full, experts=experts)
+        if hash_layer:
+            path.run_hash_layer(full, path.gate(full["x"], full["w"]))
+        else:
+            path.run(full, experts=experts)
         out_host.copy_(result_dev, non_blocking=True)
 
     one()
@@ -540,11 +587,11 @@ def measure_e2e(wl, inp, path, device, stream, steps, world, experts=None):
             "steps": steps}
 
 
-def cpu_baseline(wl, inp, budget_s: float, experts=None) -> dict:
-    n = oracle_sample_size(wl, inp, budget_s, experts)
+def cpu_baseline(wl, inp, budget_s: float, experts=None, hash_layer=False) -> dict:
+    n = oracle_sample_size(wl, inp, budget_s, experts, hash_layer)
     h = oracle_inputs(wl, inp, n, experts)
     t0 = time.perf_counter()
-    oracle_chain(wl, h)
+    oracle_chain(wl, h, hash_layer)
     dt = time.perf_counter() - t0
     return {"value": round(n / dt, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"first {n} of {wl.T} tokens of {wl.name}, full chain in fp64, "
@@ -565,21 +612,23 @@ def run_reference(args):
         experts = make_expert_weights(wl, dev)
     inp = make_inputs(wl, dev, with_y=experts is None)
     total_budget = args.cpu_budget
+    hl = bool(args.hash_layer and wl.hash_vocab)
     per_step = oracle_sample_size(wl, inp, total_budget / max(1, args.steps + args.warmup),
-                                  experts)
+                                  experts, hl)
     h = oracle_inputs(wl, inp, per_step, experts)
     for _ in range(args.warmup):
-        oracle_chain(wl, h)
+        oracle_chain(wl, h, hl)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_chain(wl, h)
+        oracle_chain(wl, h, hl)
     dt = time.perf_counter() - t0
     value = per_step * args.steps / dt
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name + ("+ffn" if experts is not None else ""),
+            "config": {"workload": (wl.name + ("+ffn" if experts is not None else "")
+                                    + ("/hash-layer" if hl else "")),
                        "tokens_per_step": per_step,
                        "parallelism": "single host core"},
             "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": 1,
@@ -606,6 +655,9 @@ def main(argv=None):
     ap.add_argument("--ffn", action="store_true",
                     help="run the experts' SwiGLU FFN (synthetic weights) on the permuted rows "
                          "instead of reading synthetic expert outputs")
+    ap.add_argument("--hash-layer", action="store_true",
+                    help="time the hash-routed layer's chain (gate, hash_route, dispatch, "
+                         "permute) of a workload that has one")
     ap.add_argument("--eager", action="store_true",
                     help="launch from the host every step instead of replaying a CUDA graph")
     ap.add_argument("--no-e2e", action="store_true")

@@ -82,3 +82,16 @@ def test_oracle_chain_with_experts_on_cpu(bench):
         f = bench.stage_flops(wl, 24)
         assert f["expert_gate_up"] == 2.0 * 24 * 2 * wl.ffn_dim * wl.d
         assert b["expert_down"] >= wl.E * wl.d * wl.ffn_dim * 2
+
+
+def test_hash_layer_chain_on_cpu(bench):
+    wl = WORKLOADS["deepseek_v4"].scaled(64)
+    import dataclasses
+    wl = dataclasses.replace(wl, d=256)  # small enough for the fp64 gate on CPU
+    inp = make_inputs(wl, "cpu", with_y=False)
+    h = bench.oracle_inputs(wl, inp, 16)
+    assert h["token_ids"].shape == (16,) and h["tid2eid"].shape == (wl.hash_vocab, wl.k_max)
+    bench.oracle_chain(wl, h, hash_layer=True)
+    b = bench.hash_stage_bytes(wl)
+    assert list(b) == ["gate_gemm", "hash_route", "dispatch", "permute"]
+    assert b["permute"] == wl.T * wl.d * 2 + wl.T * wl.k_max * wl.d * 2 + wl.T * wl.k_max * 4

@@ -65,6 +65,7 @@ __global__ void __launch_bounds__(kDispWarps * 32)
     const int64_t s = blockIdx.x;
     for (int e = lane; e < E; e += 32) hist[warp][e] = 0;
     __syncwarp();
+    griddep_wait();
     const int64_t base = (s * kDispWarps + warp) * (int64_t)items * 32;
     bool bad = false;
     for (int i0 = 0; i0 < items; i0 += kBatch) {
@@ -90,6 +91,7 @@ __global__ void __launch_bounds__(kDispWarps * 32)
         for (int w = 0; w < kDispWarps; ++w) t += hist[w][e];
         seg_total[s * E + e] = t;
     }
+    griddep_launch_dependents();
 }
 
 // A per-expert capacity and block padding (moe_dispatch_limited); the plain
@@ -122,6 +124,7 @@ __global__ void __launch_bounds__(kDispWarps * 32)
         before[e] = 0;
     }
     __syncthreads();
+    griddep_wait();
     // Lane = expert within a 32-wide chunk, warp = every 8th segment: each
     // load is a coalesced 128-byte line, and kSumUnroll of them are in flight
     // per thread before any is added.
@@ -252,6 +255,7 @@ __global__ void __launch_bounds__(kDispWarps * 32)
             __syncwarp();
         }
     }
+    griddep_launch_dependents();
 }
 
 }  // namespace
@@ -290,12 +294,19 @@ extern "C" moe_status moe_dispatch(const int32_t *topk_ids, int64_t T, int32_t k
     if (S > 0) {
         int32_t *seg_total = static_cast<int32_t *>(workspace);
         int32_t *warp_hist = seg_total + S * E;
-        dispatch_count_kernel<<<(unsigned)S, kDispWarps * 32, 0, cs>>>(topk_ids, n_flat, E, items,
-                                                                      seg_total, warp_hist,
-                                                                      d_status);
-        dispatch_scatter_kernel<false><<<(unsigned)S, kDispWarps * 32, 0, cs>>>(
-            topk_ids, n_flat, k_max, E, items, S, seg_total, warp_hist, counts, offsets,
-            sorted_token, dest_pos, Limits{INT32_MAX, 1, nullptr});
+        if (launch_pdl(dispatch_count_kernel, dim3((unsigned)S), dim3(kDispWarps * 32), 0, cs,
+                       topk_ids, n_flat, (int)E, items, seg_total, warp_hist, d_status) !=
+            cudaSuccess) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
+        if (launch_pdl(dispatch_scatter_kernel<false>, dim3((unsigned)S), dim3(kDispWarps * 32), 0,
+                       cs, topk_ids, n_flat, (int)k_max, (int)E, items, S,
+                       (const int32_t *)seg_total, (const int32_t *)warp_hist, counts, offsets,
+                       sorted_token, dest_pos, Limits{INT32_MAX, 1, nullptr}) != cudaSuccess) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
     } else {
         // No slots: every count and every offset is 0.
         if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, cs) != cudaSuccess ||
@@ -350,13 +361,20 @@ extern "C" moe_status moe_dispatch_limited(const int32_t *topk_ids, int64_t T, i
     if (S > 0) {
         int32_t *seg_total = static_cast<int32_t *>(workspace);
         int32_t *warp_hist = seg_total + S * E;
-        dispatch_count_kernel<<<(unsigned)S, kDispWarps * 32, 0, cs>>>(topk_ids, n_flat, E, items,
-                                                                      seg_total, warp_hist,
-                                                                      d_status);
+        if (launch_pdl(dispatch_count_kernel, dim3((unsigned)S), dim3(kDispWarps * 32), 0, cs,
+                       topk_ids, n_flat, (int)E, items, seg_total, warp_hist, d_status) !=
+            cudaSuccess) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
         const Limits lim{capacity > 0 ? capacity : INT32_MAX, pad, dropped};
-        dispatch_scatter_kernel<true><<<(unsigned)S, kDispWarps * 32, 0, cs>>>(
-            topk_ids, n_flat, k_max, E, items, S, seg_total, warp_hist, counts, offsets,
-            sorted_token, dest_pos, lim);
+        if (launch_pdl(dispatch_scatter_kernel<true>, dim3((unsigned)S), dim3(kDispWarps * 32), 0,
+                       cs, topk_ids, n_flat, (int)k_max, (int)E, items, S,
+                       (const int32_t *)seg_total, (const int32_t *)warp_hist, counts, offsets,
+                       sorted_token, dest_pos, lim) != cudaSuccess) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
     } else {
         if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, cs) != cudaSuccess ||
             cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), cs) != cudaSuccess ||

@@ -95,6 +95,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ int abort_s;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    griddep_wait();  // offsets and the A rows come from the kernels before this one
     const int n_tiles = a.N / a.BN;
     const int64_t total = __ldg(a.offsets + a.E);
     const int64_t m_tiles = total > 0 && total <= a.rows ? (total + kFBM - 1) / kFBM : 0;
@@ -146,6 +147,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     volatile int *abort_v = &abort_s;
+    griddep_launch_dependents();  // the next kernel may be scheduled; it waits for this grid
 
     if (warp == 0 && lane == 0) {
         // TMA producer: the stage ring runs on across tiles.
@@ -337,8 +339,11 @@ moe_status launch_expert_gemm(const moe_bf16_t *A, const moe_bf16_t *B0, const m
     // Persistent: one CTA per SM, never more CTAs than the largest tile count.
     const int64_t most = (int64_t)(a.N / a.BN) * ((rows + kFBM - 1) / kFBM);
     const int64_t grid = most < (int64_t)sm_count() ? most : (int64_t)sm_count();
-    expert_gemm_kernel<GATE_UP><<<(unsigned)grid, kFThreads, smem, as_cuda(stream)>>>(ma, mb0,
-                                                                                      mb1, a);
+    if (launch_pdl(expert_gemm_kernel<GATE_UP>, dim3((unsigned)grid), dim3(kFThreads), smem,
+                   as_cuda(stream), ma, mb0, mb1, a) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
     return launch_status();
 }
 

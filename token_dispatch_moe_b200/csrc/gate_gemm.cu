@@ -436,6 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    griddep_wait();  // inputs and outputs are free of the previous kernel
 
     if (warp == 0 && lane == 0) {
         // TMA producer.
@@ -523,6 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     tc_fence_before();
     __syncthreads();
+    griddep_launch_dependents();
     if (warp == 2) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
@@ -576,7 +578,11 @@ moe_status launch_gate(const moe_bf16_t *x, const moe_bf16_t *w, const GemmArgs 
         return MOE_ERR_CUDA;
     }
     const unsigned grid = (unsigned)((a.T + kBM - 1) / kBM);
-    gate_kernel<MODE, P, MONO, GROUPED><<<grid, kThreads, smem, as_cuda(stream)>>>(mx, mw, a, f);
+    if (launch_pdl(gate_kernel<MODE, P, MONO, GROUPED>, dim3(grid), dim3(kThreads), smem,
+                   as_cuda(stream), mx, mw, a, f) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
     return launch_status();
 }
 

@@ -487,6 +487,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const RouteArgs
     extern __shared__ __align__(128) uint8_t smem[];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
+    griddep_wait();  // the logits' producer (e.g. the gate GEMM) has completed
     const int E = a.E;
     const int R = a.R;
     const size_t stage_floats = (size_t)R * E;
@@ -574,6 +575,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const RouteArgs
             if (!mbar_wait(smem_u32(&bars[j % kStages]), (uint32_t)(j / kStages) & 1u, a.status))
                 break;
     }
+    griddep_launch_dependents();
 }
 
 template <bool VEC>
@@ -754,8 +756,10 @@ extern "C" moe_status moe_route(const float *logits, const float *bias, const in
     const int64_t cap = (int64_t)sms * per_sm;
     const unsigned grid = (unsigned)(a.ntiles < cap ? a.ntiles : cap);
     void *args[] = {&a};
-    if (cudaLaunchKernel(fn, dim3(grid), dim3(kRouteWarps * 32), args, smem, as_cuda(stream)) !=
-        cudaSuccess) {
+    cudaLaunchAttribute attr[1];
+    const cudaLaunchConfig_t cfg =
+        pdl_config(dim3(grid), dim3(kRouteWarps * 32), smem, as_cuda(stream), attr);
+    if (cudaLaunchKernelExC(&cfg, fn, args) != cudaSuccess) {
         cudaGetLastError();
         return MOE_ERR_CUDA;
     }
