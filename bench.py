@@ -145,6 +145,39 @@ def stage_flops(wl, n_assign: int) -> dict:
     return f
 
 
+def host_env(device) -> dict:
+    """What the numbers were taken on (reported, not used)."""
+    cpu = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    cpu = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    driver = None
+    try:
+        driver = subprocess.run(["nvidia-smi", "--query-gpu=driver_version", "--format=csv,noheader",
+                                 "-i", str(device.index or 0)], capture_output=True, text=True,
+                                timeout=20).stdout.strip() or None
+    except (OSError, subprocess.SubprocessError):
+        pass
+    return {"gpu": torch.cuda.get_device_name(device), "driver": driver,
+            "torch": torch.__version__, "torch_cuda": torch.version.cuda, "host_cpu": cpu,
+            "host_threads": os.cpu_count(), "seeds": "1000*workload + tensor (+100000*rank)"}
+
+
+def expert_load(counts) -> dict:
+    """Per-expert load of the routed slots and its MaxVio = (max - mean) / mean,
+    the balance measure of the aux-loss-free balancing the pages cite."""
+    c = counts.detach().cpu().double()
+    mean = float(c.mean())
+    mx = float(c.max())
+    return {"max_vio": round((mx - mean) / mean, 4) if mean > 0 else None,
+            "max_count": int(mx), "mean_count": round(mean, 2)}
+
+
 def load_peaks():
     try:
         with open(PEAKS_FILE) as f:
@@ -533,6 +566,7 @@ def run_ours(args):
                        "pad_rows_to": wl.pad, "kept_slots": limited[0],
                        "dropped_slots": n_assign - limited[0]} if limited else {})},
         "roofline": roofline, "stages": stages, "clocks": clk.summary(),
+        "load": expert_load(path.counts), "env": host_env(device),
         "gpu_launches": (5 if args.hash_layer else
                          chain_launches(wl, path.fused) + (2 if experts is not None else 0)) * K,
         "e2e": e2e,

@@ -291,6 +291,17 @@ moe_status moe_combine(const moe_bf16_t *y, const float *topk_w, const int32_t *
                        const moe_bf16_t *shared, int64_t T, int32_t k_max, int32_t d,
                        moe_bf16_t *out, moe_stream_t stream);
 
+/*
+ * moe_wait_probe -- diagnostic (no counterpart in the pages): one warp runs the
+ * library's bounded mbarrier wait against a barrier that nothing completes,
+ * with a limit of limit_ns nanoseconds (1 ns .. 1 s).  The wait gives up,
+ * *d_status receives MOE_ERR_TIMEOUT (first error wins) and *d_outcome
+ * (nullable) 2 (1 would mean the barrier completed).  Lets a test exercise the
+ * timeout path every kernel's waits take, with no fault and no hang.
+ */
+moe_status moe_wait_probe(uint64_t limit_ns, int32_t *d_status, int32_t *d_outcome,
+                          moe_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * Expert-parallel exchange.  In multi-GPU expert parallelism every router
  * choice becomes all-to-all traffic ("I modelli MoE open hanno router

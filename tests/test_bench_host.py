@@ -95,3 +95,10 @@ def test_hash_layer_chain_on_cpu(bench):
     b = bench.hash_stage_bytes(wl)
     assert list(b) == ["gate_gemm", "hash_route", "dispatch", "permute"]
     assert b["permute"] == wl.T * wl.d * 2 + wl.T * wl.k_max * wl.d * 2 + wl.T * wl.k_max * 4
+
+
+def test_expert_load_max_vio(bench):
+    import torch
+    r = bench.expert_load(torch.tensor([1, 1, 1, 5], dtype=torch.int32))
+    assert r == {"max_vio": 1.5, "max_count": 5, "mean_count": 2.0}
+    assert bench.expert_load(torch.tensor([3, 3, 3], dtype=torch.int32))["max_vio"] == 0.0

@@ -530,3 +530,24 @@ def test_route_grouped_validation():
         p = moe.RouteParams.make(E_, k, "softmax", G, 1, 1, True, 1.0)
         with pytest.raises((moe.MoeError, ValueError)):
             moe.moe_route_grouped(logits, p, kpg, ids[:, :k].contiguous(), w[:, :k].contiguous())
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    """The wait every kernel uses gives up on a barrier that nothing completes,
+    records MOE_ERR_TIMEOUT and returns; the next calls run normally."""
+    st = _status()
+    outcome = torch.zeros((1,), dtype=torch.int32, device=DEV)
+    moe.moe_wait_probe(20_000_000, st, outcome)  # 20 ms
+    torch.cuda.synchronize()
+    assert st.item() == moe.MOE_ERR_TIMEOUT and outcome.item() == 2
+    with pytest.raises(moe.MoeError):
+        moe.moe_wait_probe(0, st)
+    logits = torch.randn((64, 16), generator=_gen(5), device=DEV)
+    p = moe.RouteParams.make(16, 2, "softmax")
+    ids = torch.empty((64, 2), dtype=torch.int32, device=DEV)
+    w = torch.empty((64, 2), device=DEV)
+    st2 = _status()
+    moe.moe_route(logits, None, None, p, ids, w, st2)
+    torch.cuda.synchronize()
+    assert st2.item() == 0
+    assert torch.equal(ids[:, 0], logits.argmax(dim=1).to(torch.int32))

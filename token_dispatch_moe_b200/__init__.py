@@ -89,6 +89,7 @@ def load_library(path: str | None = None):
         "moe_dispatch_static": ([P, i64, i32, i32, P, P, P, P, P, P], st),
         "moe_expert_gate_up": ([P, P, P, P, P, P, i32, i32, i32, i64, i32, P, P, P], st),
         "moe_expert_down": ([P, P, P, P, i32, i32, i32, i64, P, P, P], st),
+        "moe_wait_probe": ([ctypes.c_uint64, P, P, P], st),
         "moe_route_grouped": ([P, ctypes.POINTER(RouteParams), i32, i64, P, P, P, P], st),
         "moe_ep_layout": ([P, P, P, P, i32, i32, i64, i32, i32, P, P, P, P, P], st),
         "moe_ep_permute": ([P, P, P, P, i32, i64, i64, i32, i32, P, P], st),
@@ -387,6 +388,15 @@ def moe_expert_down(h, offsets, w2, y, b2=None, d_status=None, stream=None):
     _check(load_library().moe_expert_down(_ptr(h), _ptr(offsets), _ptr(w2), _ptr(b2), E, d, F,
                                           rows, _ptr(y), _ptr(d_status), _stream(stream)),
            "moe_expert_down")
+
+
+def moe_wait_probe(limit_ns: int, d_status, d_outcome=None, stream=None):
+    """Run the library's bounded wait against a barrier nothing completes (a
+    diagnostic for the timeout path): *d_status gets MOE_ERR_TIMEOUT."""
+    _need(d_status, torch.int32, "d_status")
+    _need(d_outcome, torch.int32, "d_outcome")
+    _check(load_library().moe_wait_probe(limit_ns, _ptr(d_status), _ptr(d_outcome),
+                                         _stream(stream)), "moe_wait_probe")
 
 
 def moe_dispatch_static(topk_ids, E, counts, offsets, sorted_token, dest_pos, d_status=None,

@@ -32,6 +32,7 @@
 //    chunks, a group's top-2 is merged with register shuffles; otherwise each
 //    lane scans a strip of the group in shared memory.
 #include "common.cuh"
+#include "tc.cuh"
 
 namespace moe {
 namespace {
@@ -39,7 +40,6 @@ namespace {
 constexpr int kRouteWarps = 8;  // warps per block
 constexpr int kMaxE = 512;
 constexpr int kStages = 3;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 struct RouteArgs {
     const float *logits;
@@ -61,40 +61,6 @@ struct RouteArgs {
 };
 
 // ---------------------------------------------------------------- helpers --
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ uint64_t global_timer_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t *status) {
-    if (mbar_try(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try(bar, parity)) return true;
-        if ((it & 255u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) {
-            report(status, MOE_ERR_TIMEOUT);
-            return false;
-        }
-    }
-}
-
 // Copies `bytes` (a multiple of 16, may be 0) from global src to shared dst;
 // completion is counted on the mbarrier's transaction count.
 __device__ __forceinline__ void bulk_copy(uint32_t dst, const void *src, uint32_t bytes,

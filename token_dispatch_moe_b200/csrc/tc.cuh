@@ -35,17 +35,23 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase of the given parity; false (and a recorded
-// MOE_ERR_TIMEOUT) if it has not completed within the limit.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t *status) {
+// MOE_ERR_TIMEOUT) if it has not completed within limit_ns of %globaltimer.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, int32_t *status,
+                                              uint64_t limit_ns) {
     if (mbar_try(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try(bar, parity)) return true;
-        if ((it & 255u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) {
+        if ((it & 255u) == 0u && global_timer_ns() - t0 > limit_ns) {
             report(status, MOE_ERR_TIMEOUT);
             return false;
         }
     }
+}
+
+// The library's waits: about 2 s, far above any copy or MMA they wait for.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t *status) {
+    return mbar_wait_for(bar, parity, status, kWaitLimitNs);
 }
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
