@@ -559,7 +559,9 @@ moe_status plan_gemm(int64_t T, int32_t d, int32_t E, size_t epi_bytes, GemmArgs
         return MOE_ERR_CUDA;
     }
     const int overhead = 1024 + 256;  // alignment slack + barriers and TMEM slot
-    int stages = (int)((max_smem - overhead - (int64_t)epi_bytes) / (int)a.stage_bytes);
+    const int static_smem = 1024;     // the kernel's own __shared__ alignment block
+    int stages = (int)((max_smem - static_smem - overhead - (int64_t)epi_bytes) /
+                       (int)a.stage_bytes);
     if (stages > 8) stages = 8;
     if (stages < 2) return MOE_ERR_UNSUPPORTED;
     a.stages = stages;
