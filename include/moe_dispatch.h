@@ -12,6 +12,18 @@
  *   moe_combine    -> weighted fp32 sum of expert outputs back in token order,
  *                     plus an optional shared expert
  *
+ * Further entry points on the same buffers:
+ *   moe_gate_route            gate GEMM with the route in its epilogue
+ *   moe_route_grouped         per-group candidates, then a global top-k
+ *   moe_dispatch_limited      dispatch with a per-expert capacity and expert
+ *                             blocks padded for tiled expert GEMMs
+ *   moe_expert_gate_up / moe_expert_down
+ *                             the routed experts' SwiGLU FFN (grouped GEMMs)
+ *   moe_ep_layout / moe_ep_permute / moe_ep_combine
+ *                             expert-parallel exchange over peer memory
+ *   moe_dispatch_static       dispatch without a caller workspace
+ *   moe_wait_probe            diagnostic for the bounded-wait timeout path
+ *
  * Conventions shared by every entry point:
  *   - All tensor pointers are DEVICE pointers into memory the caller owns; the
  *     library never allocates, frees or synchronises, and launches only on the

@@ -37,7 +37,7 @@ constexpr int kMaxPad = 4096;   // largest block padding of moe_dispatch_limited
 
 int warp_items(int64_t n_flat) {
     int items = 4;
-    while ((int64_t)items * 32 * kDispWarps * 148 < n_flat && items < 64) items *= 2;
+    while ((int64_t)items * 32 * kDispWarps * 148 < n_flat && items < 16) items *= 2;
     return items;
 }
 

@@ -11,7 +11,9 @@
 // over destination rows would re-read x k times) with streaming stores, which
 // measured 3 % faster than plain ones for the permuted rows.  combine gathers the k_t
 // expert rows of a token and writes one row; loads of four slots are issued
-// before their FMAs so that enough bytes are in flight per warp.
+// before their FMAs so that enough bytes are in flight per warp (four vectors
+// per lane per slot where the row has them: at d = 2048 that took combine from
+// 104.6 to 102.2 us against two).
 #include "common.cuh"
 #include "rows.cuh"
 
@@ -143,8 +145,21 @@ extern "C" moe_status moe_combine(const moe_bf16_t *y, const float *topk_w,
     if (!out || !aligned16(out) || (shared && !aligned16(shared))) return MOE_ERR_INVALID_ARG;
     if (k_max > 0 && (!y || !topk_w || !dest_pos || !aligned16(y))) return MOE_ERR_INVALID_ARG;
     if (T * (int64_t)k_max >= (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
-    combine_kernel<2><<<row_grid(T), kRowWarps * 32, 0, as_cuda(stream)>>>(
-        reinterpret_cast<const uint4 *>(y), topk_w, dest_pos,
-        reinterpret_cast<const uint4 *>(shared), T, k_max, d / 8, reinterpret_cast<uint4 *>(out));
+    // Vectors per lane per slot: as many as the row has for the whole warp, up
+    // to four (short rows would leave lanes idle).
+    const int nvec = d / 8;
+    const uint4 *y4 = reinterpret_cast<const uint4 *>(y);
+    const uint4 *s4 = reinterpret_cast<const uint4 *>(shared);
+    uint4 *o4 = reinterpret_cast<uint4 *>(out);
+    const unsigned grid = row_grid(T);
+    if (nvec >= 128)
+        combine_kernel<4><<<grid, kRowWarps * 32, 0, as_cuda(stream)>>>(y4, topk_w, dest_pos, s4,
+                                                                        T, k_max, nvec, o4);
+    else if (nvec >= 64)
+        combine_kernel<2><<<grid, kRowWarps * 32, 0, as_cuda(stream)>>>(y4, topk_w, dest_pos, s4,
+                                                                        T, k_max, nvec, o4);
+    else
+        combine_kernel<1><<<grid, kRowWarps * 32, 0, as_cuda(stream)>>>(y4, topk_w, dest_pos, s4,
+                                                                        T, k_max, nvec, o4);
     return launch_status();
 }

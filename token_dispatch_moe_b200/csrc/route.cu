@@ -265,11 +265,12 @@ extern "C" moe_status moe_route(const float *logits, const float *bias, const in
     RouteArgs a;
     fill_route_args(a, logits, bias, k_per_token, *p, T, topk_ids, topk_w, d_status);
     const bool vec = (E % 4 == 0);
-    // Rows per tile: about 16 KB of logits, but small enough that every SM
-    // gets at least two tiles (each row is a serial chain of warp reductions,
-    // so small batches need the rows spread out).
+    // Rows per tile: about 8 KB of logits (16 KB for top-1, whose rows are
+    // short), and small enough that every SM gets at least two tiles (each row
+    // is a serial chain of warp reductions, so the rows are spread over as
+    // many resident warps as possible).
     const int sms = sm_count();
-    int R = (4096 / E) / 8 * 8;
+    int R = ((p->k_max == 1 && G == 1 ? 4096 : 2048) / E) / 8 * 8;
     const int64_t spread = ((T + 2 * sms - 1) / (2 * sms) + 7) / 8 * 8;
     if (spread < R) R = (int)spread;
     R = R < 8 ? 8 : (R > 256 ? 256 : R);
