@@ -145,3 +145,50 @@ def test_ep_validation():
                           torch.zeros((10, 2), dtype=torch.int32, device=DEV), rs.dest_pos,
                           rs.offsets, 0, rs.dest_rank, rs.dest_row,
                           torch.zeros((4,), dtype=torch.int32, device=DEV))
+
+
+def test_ep_step_one_rank_over_nccl():
+    """The whole exchange step of ep.py (count all-gather and barriers over
+    NCCL, layout, peer stores, experts, peer loads) on a one-rank group, with
+    plain device buffers standing in for the symmetric ones."""
+    import socket
+
+    import torch.distributed as dist
+
+    from token_dispatch_moe_b200.ep import ep_step
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            device_id=torch.device(DEV, torch.cuda.current_device()))
+    try:
+        T, k, E, d = 500, 4, 16, 256
+        xs, ids, ws, sh = _ranks_inputs(1, T, k, E, d, 123)
+        rs = EpRank(T, k, E, 1, 0)
+        cap = T * k
+        recv = torch.zeros((cap, d), dtype=torch.bfloat16, device=DEV)
+        y = torch.zeros((cap, d), dtype=torch.bfloat16, device=DEV)
+        out = torch.empty((T, d), dtype=torch.bfloat16, device=DEV)
+
+        def experts(recv_buf, y_buf, recv_offsets):
+            y_buf.copy_(recv_buf)  # identity experts
+
+        all_counts = ep_step(rs, xs[0], ids[0], ws[0], sh[0], out, recv, moe.peer_table([recv]), y,
+                             moe.peer_table([y]), experts)
+        torch.cuda.synchronize()
+        assert rs.status.item() == 0
+        flat = ids[0].reshape(-1)
+        assert torch.equal(all_counts[0], torch.bincount(flat[flat >= 0].long(), minlength=E)
+                           .to(torch.int32))
+        lay = oracle.ep_layout(ids[0].cpu().numpy()[None], E)
+        o = oracle.ep_combine([bits(recv[:int(lay["recv_rows"][0])])], ws[0].cpu().numpy()[None],
+                              lay["dest_rank"], lay["dest_row"], bits(sh[0])[None])
+        ref, mag = o[0]
+        got = bits_to_f64(bits(out))
+        assert np.all(np.abs(got - ref) <= 1e-2 * np.maximum(np.abs(ref), mag))
+        # identity experts: the received rows are the tokens' own rows
+        want = oracle.ep_permute(bits(xs[0])[None], lay["dest_rank"], lay["dest_row"],
+                                 lay["recv_rows"])
+        assert np.array_equal(bits(recv[:int(lay["recv_rows"][0])]), want[0])
+    finally:
+        dist.destroy_process_group()

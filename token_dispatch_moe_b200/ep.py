@@ -11,7 +11,7 @@ from __future__ import annotations
 import torch
 
 from . import moe_dispatch, moe_dispatch_workspace_size, moe_ep_combine, moe_ep_layout, \
-    moe_ep_permute, peer_table
+    moe_ep_permute
 
 
 def experts_per_rank(E: int, G: int) -> int:
