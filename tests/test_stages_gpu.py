@@ -251,7 +251,8 @@ def test_dispatch_edge_cases():
 @pytest.mark.parametrize("T,k,E,cap,pad,hot", [
     (1, 1, 4, 0, 1, False), (3001, 1, 128, 0, 128, True), (70000, 1, 128, 547, 128, True),
     (5000, 8, 64, 400, 16, False), (777, 6, 384, 3, 1, True), (40000, 4, 128, 1, 7, True),
-    (20000, 16, 512, 0, 64, False), (9000, 2, 8, 2250, 128, True)])
+    (20000, 16, 512, 0, 64, False), (9000, 2, 8, 2250, 128, True),
+    (200, 2, 8, 0, 4096, False), (3000, 32, 16, 5, 1, True)])
 def test_dispatch_limited_parity(T, k, E, cap, pad, hot):
     """Capacity cut and block padding, bit-exact against the oracle."""
     g = _gen(T * 7 + E + cap + pad)
