@@ -168,6 +168,27 @@ def host_env(device) -> dict:
             "host_threads": os.cpu_count(), "seeds": "1000*workload + tensor (+100000*rank)"}
 
 
+def launch_floor_us(device, stream, reps: int = 200) -> float:
+    """Device time of a one-element kernel replayed from a CUDA graph on the
+    bench's stream: the floor under any single stage's time."""
+    t = torch.zeros((1,), device=device)
+    cap = torch.cuda.Stream(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        t.add_(1.0)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    del g
+    return round(us, 2)
+
+
 def expert_load(counts) -> dict:
     """Per-expert load of the routed slots and its MaxVio = (max - mean) / mean,
     the balance measure of the aux-loss-free balancing the pages cite."""
@@ -511,6 +532,8 @@ def run_ours(args):
     step_ms = [m[-1] for m in marks]
     stage_ms = {n: statistics.fmean(m[i + 1] - m[i] for m in marks) for i, n in enumerate(names)}
     ms = statistics.fmean(step_ms)
+    srt = sorted(step_ms)
+    ms_p50, ms_p90 = srt[len(srt) // 2], srt[min(len(srt) - 1, (9 * len(srt)) // 10)]
     ms_max = reduce_max(ms, world, device)
     value = job_throughput(wl.T, world, ms_max / 1e3)
 
@@ -554,6 +577,8 @@ def run_ours(args):
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_max, 5),
+        "ms_p50": round(ms_p50, 5), "ms_p90": round(ms_p90, 5),
+        "launch_floor_us": launch_floor_us(device, stream),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
         "data": "synthetic",
         "config": {"workload": (wl.name + ("+ffn" if experts is not None else "")
