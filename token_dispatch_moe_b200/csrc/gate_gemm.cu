@@ -564,6 +564,20 @@ moe_status plan_gemm(int64_t T, int32_t d, int32_t E, size_t epi_bytes, GemmArgs
                        (int)a.stage_bytes);
     if (stages > 8) stages = 8;
     if (stages < 2) return MOE_ERR_UNSUPPORTED;
+    // More tiles than SMs (several waves), a plain epilogue and at most half of
+    // the TMEM: two CTAs per SM, so that one's epilogue and pipeline fill
+    // overlap the other's mainloop (deepseek_v3's gate: 328 -> 253 us), with
+    // as many stages as half of the SM's shared memory holds.
+    const int64_t tiles = (T + kBM - 1) / kBM;
+    int per_sm_smem = 0;
+    if (epi_bytes == 0 && a.tmem_cols <= 256 && tiles > sm_count() &&
+        cudaDeviceGetAttribute(&per_sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) ==
+            cudaSuccess) {
+        const int half = per_sm_smem / 2 - 1024;  // 1 KB per block is reserved by the system
+        const int s2 = (half - static_smem - overhead) / (int)a.stage_bytes;
+        if (s2 >= 2) stages = s2 < stages ? s2 : stages;
+    }
+    cudaGetLastError();
     a.stages = stages;
     smem = (size_t)stages * a.stage_bytes + overhead + epi_bytes;
     return MOE_OK;
