@@ -54,6 +54,24 @@ def test_gate_gemm_random(T, d, E):
     check_gate(logits, x, w)
 
 
+@pytest.mark.parametrize("T,d,E", [(20000, 512, 384), (19500, 256, 300), (40000, 256, 256),
+                                   (30001, 128, 128)])
+def test_gate_gemm_several_waves(T, d, E):
+    """More tiles than SMs (two CTAs per SM where the accumulator takes at most
+    half the TMEM): every logit is written, and sampled rows (the first and
+    last tiles included) match the oracle."""
+    g = _gen(T + d + E)
+    x = torch.randn((T, d), generator=g, device=DEV).to(torch.bfloat16)
+    w = (torch.randn((E, d), generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    logits = torch.full((T, E), float("nan"), device=DEV)
+    moe.moe_gate_gemm(x, w, logits)
+    torch.cuda.synchronize()
+    assert not torch.isnan(logits).any()
+    rows = np.unique(np.concatenate([np.arange(130), np.arange(T - 130, T),
+                                     np.random.default_rng(T).choice(T, 600, replace=False)]))
+    check_gate(logits, x, w, rows)
+
+
 def test_gate_gemm_validation():
     x = torch.zeros((4, 12), dtype=torch.bfloat16, device=DEV)
     w = torch.zeros((4, 12), dtype=torch.bfloat16, device=DEV)
