@@ -500,15 +500,33 @@ def run_ours(args):
             if err != 0:
                 raise RuntimeError(f"cudaEventRecordWithFlags failed ({err})")
 
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=cap, capture_error_mode="relaxed"):
-            run_step(mark)
-        graph.replay()
-        torch.cuda.synchronize()
-        times = []
+        def make_graph(every_stage):
+            # An event node between two kernels replaces their programmatic
+            # (PDL) edge by a full dependency, so the timed step carries events
+            # at its two ends only; a second graph of the same step marks every
+            # stage boundary for the per-stage breakdown.
+            def m(i):
+                if every_stage or i in (0, nb - 1):
+                    mark(i)
+
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap, capture_error_mode="relaxed"):
+                run_step(m)
+            g.replay()
+            torch.cuda.synchronize()
+            return g
+
+        graph = make_graph(False)
+        graph_stages = make_graph(True)
+        step_times, times = [], []
 
         def timed_step(s):
             graph.replay()
+            torch.cuda.synchronize()
+            step_times.append(gev[0].elapsed_time(gev[nb - 1]))
+
+        def stage_step(s):
+            graph_stages.replay()
             torch.cuda.synchronize()
             times.append([gev[0].elapsed_time(gev[i]) for i in range(nb)])
 
@@ -525,11 +543,17 @@ def run_ours(args):
             timed_step(s)
         torch.cuda.synchronize()
         barrier(world, device)
+        if not args.eager:
+            for s in range(K):  # the per-stage breakdown, after the timed region
+                flush.zero_()
+                stage_step(s)
+            torch.cuda.synchronize()
     if args.eager:
         marks = [[evs[s][0].elapsed_time(evs[s][i]) for i in range(nb)] for s in range(K)]
+        step_ms = [m[-1] for m in marks]
     else:
         marks = times
-    step_ms = [m[-1] for m in marks]
+        step_ms = step_times
     stage_ms = {n: statistics.fmean(m[i + 1] - m[i] for m in marks) for i, n in enumerate(names)}
     ms = statistics.fmean(step_ms)
     srt = sorted(step_ms)
@@ -596,7 +620,12 @@ def run_ours(args):
                    **({"capacity": path.capacity, "capacity_factor": wl.capacity_factor,
                        "pad_rows_to": wl.pad, "kept_slots": limited[0],
                        "dropped_slots": n_assign - limited[0]} if limited else {})},
-        "roofline": roofline, "stages": stages, "clocks": clk.summary(),
+        "roofline": roofline, "stages": stages,
+        "stages_timed": ("events on the stream around each stage" if args.eager else
+                         "a second graph of the step with an event node at every stage "
+                         "boundary, replayed K times after the timed region"),
+        "ms_per_step_stage_marked": round(statistics.fmean(m[-1] for m in marks), 5),
+        "clocks": clk.summary(),
         "load": expert_load(path.counts), "env": host_env(device),
         "gpu_launches": (5 if args.hash_layer else
                          chain_launches(wl, path.fused) + (2 if experts is not None else 0)) * K,

@@ -48,7 +48,7 @@ def test_static_scratch_matches_workspace_dispatch(T, k, E):
 
 
 def test_static_scratch_refuses_oversize():
-    T, k, E = 262144, 32, 512  # needs more than the fixed 4 MiB
+    T, k, E = 524288, 32, 512  # needs more than the fixed 4 MiB
     assert moe.moe_dispatch_workspace_size(T, k, E) > 4 << 20
     ids = torch.zeros((T, k), dtype=torch.int32, device=DEV)
     out = _outputs(T, k, E)

@@ -7,21 +7,22 @@
 // dest_pos[a] = pos (-1 for empty slots).
 //
 // B200 design: two short launches, no inter-block waiting.  The slots are cut
-// into S block segments of 8 warps x W items x 32 lanes, each warp owning a
+// into S block segments of 8 warps x ITEMS items x 32 lanes, each warp owning a
 // contiguous sub-segment.
-//   1. count:   every warp builds its sub-segment's histogram in shared memory
+//   1. count:   every block builds its segment's histogram in shared memory
 //               with warp-aggregated updates (__match_any_sync: one leader per
-//               distinct id adds the popcount of its peers) and stores it; the
-//               block also stores its segment's total per expert.
-//   2. scatter: each block sums the segment totals of the whole grid (all S,
-//               for counts; those before it, for its own base) straight from
-//               L2, scans counts into offsets (block 0 writes counts and
-//               offsets), adds the per-warp histograms of the earlier warps of
-//               its segment, then every warp walks its sub-segment again in
-//               order, ranks each slot among its peers with the same id
-//               (popcount of lower lanes in the match mask) and writes
+//               distinct id adds the popcount of its peers) and stores it.
+//   2. scatter: every warp loads its sub-segment's ids into registers while
+//               the block loads the segment totals of the whole grid (16-byte
+//               loads, all in flight together), so the kernel waits on memory
+//               once.  The block sums all S totals (for counts) and those
+//               before it (for its own base), scans counts into offsets
+//               (block 0 writes counts and offsets), rebuilds its warps'
+//               histograms from the ids in registers, and every warp walks
+//               its ids in order, ranking each slot among its peers with the
+//               same id (popcount of lower lanes in the match mask), writing
 //               sorted_token and dest_pos.
-// Workspace: seg_total [S][E] and warp_hist [S][8][E], int32.
+// Workspace: seg_total [S][Ep] int32, Ep = E rounded up to a multiple of 4.
 #include <atomic>
 
 #include "common.cuh"
@@ -31,8 +32,7 @@ namespace {
 
 constexpr int kDispWarps = 8;
 constexpr int kMaxE = 512;
-constexpr int kBatch = 4;  // slot loads issued together per lane (items is a multiple)
-constexpr int kSumUnroll = 16;  // independent segment-total loads in flight per thread
+constexpr int kSumUnroll = 16;  // independent 16-byte segment-total loads in flight per thread
 constexpr int kMaxPad = 4096;   // largest block padding of moe_dispatch_limited
 
 int warp_items(int64_t n_flat) {
@@ -46,6 +46,9 @@ int64_t num_segments(int64_t n_flat, int items) {
     return (n_flat + seg - 1) / seg;
 }
 
+// Row stride of seg_total: whole 16-byte quads per segment.
+int seg_stride(int E) { return (E + 3) / 4 * 4; }
+
 __device__ __forceinline__ int load_id(const int32_t *ids, int64_t a, int64_t n_flat, int E,
                                        bool &bad) {
     int e = a < n_flat ? ids[a] : -1;
@@ -56,41 +59,30 @@ __device__ __forceinline__ int load_id(const int32_t *ids, int64_t a, int64_t n_
     return e;
 }
 
+template <int ITEMS>
 __global__ void __launch_bounds__(kDispWarps * 32)
-    dispatch_count_kernel(const int32_t *__restrict__ ids, int64_t n_flat, int E, int items,
-                          int32_t *__restrict__ seg_total, int32_t *__restrict__ warp_hist,
-                          int32_t *status) {
-    __shared__ int32_t hist[kDispWarps][kMaxE];
+    dispatch_count_kernel(const int32_t *__restrict__ ids, int64_t n_flat, int E, int Ep,
+                          int32_t *__restrict__ seg_total, int32_t *status) {
+    __shared__ int32_t hist[kMaxE];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t s = blockIdx.x;
-    for (int e = lane; e < E; e += 32) hist[warp][e] = 0;
-    __syncwarp();
+    for (int e = threadIdx.x; e < Ep; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
     griddep_wait();
-    const int64_t base = (s * kDispWarps + warp) * (int64_t)items * 32;
+    const int64_t base = (s * kDispWarps + warp) * (int64_t)ITEMS * 32;
     bool bad = false;
-    for (int i0 = 0; i0 < items; i0 += kBatch) {
-        int eb[kBatch];  // loads of a batch are issued before any of them is used
+    int eb[ITEMS];  // every load of the sub-segment is issued before any is used
 #pragma unroll
-        for (int j = 0; j < kBatch; ++j)
-            eb[j] = load_id(ids, base + (int64_t)(i0 + j) * 32 + lane, n_flat, E, bad);
+    for (int j = 0; j < ITEMS; ++j) eb[j] = load_id(ids, base + (int64_t)j * 32 + lane, n_flat, E, bad);
 #pragma unroll
-        for (int j = 0; j < kBatch; ++j) {
-            const int e = eb[j];
-            const unsigned peers = __match_any_sync(MOE_FULL_MASK, e);
-            if (e >= 0 && lane == __ffs(peers) - 1) hist[warp][e] += __popc(peers);
-            __syncwarp();
-        }
+    for (int j = 0; j < ITEMS; ++j) {
+        const int e = eb[j];
+        const unsigned peers = __match_any_sync(MOE_FULL_MASK, e);
+        if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[e], __popc(peers));
     }
     if (__any_sync(MOE_FULL_MASK, bad) && lane == 0) report(status, MOE_ERR_DEVICE_INDEX);
-    int32_t *wh = warp_hist + (s * kDispWarps + warp) * E;
-    for (int e = lane; e < E; e += 32) wh[e] = hist[warp][e];
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int32_t t = 0;
-#pragma unroll
-        for (int w = 0; w < kDispWarps; ++w) t += hist[w][e];
-        seg_total[s * E + e] = t;
-    }
+    for (int e = threadIdx.x; e < Ep; e += blockDim.x) seg_total[s * Ep + e] = hist[e];
     griddep_launch_dependents();
 }
 
@@ -102,52 +94,87 @@ struct Limits {
     int32_t *dropped;  // nullable: number of slots over capacity
 };
 
-template <bool LIMITED>
+template <int ITEMS, bool LIMITED>
 __global__ void __launch_bounds__(kDispWarps * 32)
     dispatch_scatter_kernel(const int32_t *__restrict__ ids, int64_t n_flat, int k_max, int E,
-                            int items, int64_t S, const int32_t *__restrict__ seg_total,
-                            const int32_t *__restrict__ warp_hist, int32_t *__restrict__ counts,
-                            int32_t *__restrict__ offsets, int32_t *__restrict__ sorted_token,
-                            int32_t *__restrict__ dest_pos, Limits lim) {
-    __shared__ int32_t total[kMaxE + 1];
+                            int Ep, int64_t S, const int32_t *__restrict__ seg_total,
+                            int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+                            int32_t *__restrict__ sorted_token, int32_t *__restrict__ dest_pos,
+                            Limits lim) {
+    __shared__ int32_t total[kMaxE];
     __shared__ int32_t before[kMaxE];
-    __shared__ int32_t run[kDispWarps][kMaxE];
+    __shared__ int32_t hist[kDispWarps][kMaxE];
     __shared__ int32_t wsum[kDispWarps];
     __shared__ int32_t kept_s[LIMITED ? kMaxE : 1];
     __shared__ int32_t drop_s;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t s = blockIdx.x;
 
-    // Per-expert totals over all segments and over the segments before this one.
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    for (int e = threadIdx.x; e < Ep; e += blockDim.x) {
         total[e] = 0;
         before[e] = 0;
     }
+    for (int i = threadIdx.x; i < kDispWarps * Ep; i += blockDim.x) hist[i / Ep][i % Ep] = 0;
     __syncthreads();
     griddep_wait();
-    // Lane = expert within a 32-wide chunk, warp = every 8th segment: each
-    // load is a coalesced 128-byte line, and kSumUnroll of them are in flight
-    // per thread before any is added.
-    for (int c = 0; c < E; c += 32) {
-        const int e = c + lane;
-        int32_t acc_t = 0, acc_b = 0;
-        for (int64_t sp0 = warp; sp0 < S; sp0 += (int64_t)kDispWarps * kSumUnroll) {
-            int32_t v[kSumUnroll];
+
+    // This warp's ids: loaded once, kept in registers for both passes below.
+    const int64_t base = (s * kDispWarps + warp) * (int64_t)ITEMS * 32;
+    bool bad = false;
+    int eb[ITEMS];
 #pragma unroll
-            for (int u = 0; u < kSumUnroll; ++u) {
-                const int64_t sp = sp0 + (int64_t)u * kDispWarps;
-                v[u] = (e < E && sp < S) ? seg_total[sp * E + e] : 0;
-            }
+    for (int j = 0; j < ITEMS; ++j) eb[j] = load_id(ids, base + (int64_t)j * 32 + lane, n_flat, E, bad);
+
+    // Per-expert totals over all segments and over the segments before this
+    // one.  Thread = (quad q of 4 experts, segment residue r); nsr residues
+    // walk the segments in steps of nsr, kSumUnroll 16-byte loads in flight.
+    {
+        const int Q = Ep / 4;
+        const int nsr = (int)blockDim.x / Q;
+        const int q = (int)threadIdx.x % Q, r = (int)threadIdx.x / Q;
+        if (r < nsr) {
+            const int4 *st4 = reinterpret_cast<const int4 *>(seg_total);
+            int4 at = make_int4(0, 0, 0, 0), ab = make_int4(0, 0, 0, 0);
+            for (int64_t sp0 = r; sp0 < S; sp0 += (int64_t)nsr * kSumUnroll) {
+                int4 v[kSumUnroll];
 #pragma unroll
-            for (int u = 0; u < kSumUnroll; ++u) {
-                acc_t += v[u];
-                acc_b += (sp0 + (int64_t)u * kDispWarps < s) ? v[u] : 0;
+                for (int u = 0; u < kSumUnroll; ++u) {
+                    const int64_t sp = sp0 + (int64_t)u * nsr;
+                    v[u] = sp < S ? st4[sp * Q + q] : make_int4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int u = 0; u < kSumUnroll; ++u) {
+                    at.x += v[u].x;
+                    at.y += v[u].y;
+                    at.z += v[u].z;
+                    at.w += v[u].w;
+                    if (sp0 + (int64_t)u * nsr < s) {
+                        ab.x += v[u].x;
+                        ab.y += v[u].y;
+                        ab.z += v[u].z;
+                        ab.w += v[u].w;
+                    }
+                }
             }
+            atomicAdd(&total[4 * q + 0], at.x);
+            atomicAdd(&total[4 * q + 1], at.y);
+            atomicAdd(&total[4 * q + 2], at.z);
+            atomicAdd(&total[4 * q + 3], at.w);
+            atomicAdd(&before[4 * q + 0], ab.x);
+            atomicAdd(&before[4 * q + 1], ab.y);
+            atomicAdd(&before[4 * q + 2], ab.z);
+            atomicAdd(&before[4 * q + 3], ab.w);
         }
-        if (e < E) {
-            atomicAdd(&total[e], acc_t);
-            atomicAdd(&before[e], acc_b);
-        }
+    }
+
+    // This warp's histogram, from the ids in registers (one leader per id).
+    unsigned pm[ITEMS];
+#pragma unroll
+    for (int j = 0; j < ITEMS; ++j) {
+        const int e = eb[j];
+        pm[j] = __match_any_sync(MOE_FULL_MASK, e);
+        if (e >= 0 && lane == __ffs(pm[j]) - 1) hist[warp][e] += __popc(pm[j]);
+        __syncwarp();
     }
     __syncthreads();
 
@@ -198,8 +225,6 @@ __global__ void __launch_bounds__(kDispWarps * 32)
                 if (LIMITED && lim.dropped) *lim.dropped = drop_s;
             }
         }
-        // Each warp's starting position per expert: offset + earlier segments +
-        // earlier warps of this segment.
         __syncthreads();
         if (i0 < E) total[i0] = excl;
         if (i1 < E) total[i1] = excl + c0;
@@ -214,48 +239,67 @@ __global__ void __launch_bounds__(kDispWarps * 32)
                 sorted_token[p] = -1;
         }
     }
-    // Each warp's first rank per expert (earlier segments + earlier warps of
-    // this segment); without limits the block offset is folded in as well.
-    const int32_t *wh = warp_hist + s * kDispWarps * E;
-    int32_t *r = run[warp];
-    for (int e = lane; e < E; e += 32) {
-        int32_t v[kDispWarps];
-#pragma unroll
-        for (int w = 0; w < kDispWarps; ++w) v[w] = w < warp ? wh[w * E + e] : 0;
+    // Each warp's first rank per expert, in place of its histogram: earlier
+    // segments + earlier warps of this segment; without limits the block
+    // offset is folded in as well.
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int32_t b = (LIMITED ? 0 : total[e]) + before[e];
 #pragma unroll
-        for (int w = 0; w < kDispWarps; ++w) b += v[w];
-        r[e] = b;
-    }
-    __syncwarp();
-
-    const int64_t base = (s * kDispWarps + warp) * (int64_t)items * 32;
-    const unsigned lower = (1u << lane) - 1u;
-    bool bad = false;
-    for (int i0 = 0; i0 < items; i0 += kBatch) {
-        int eb[kBatch];
-#pragma unroll
-        for (int j = 0; j < kBatch; ++j)
-            eb[j] = load_id(ids, base + (int64_t)(i0 + j) * 32 + lane, n_flat, E, bad);
-#pragma unroll
-        for (int j = 0; j < kBatch; ++j) {
-            const int64_t a = base + (int64_t)(i0 + j) * 32 + lane;
-            const int e = eb[j];
-            const unsigned peers = __match_any_sync(MOE_FULL_MASK, e);
-            if (e >= 0) {
-                int32_t pos = r[e] + __popc(peers & lower);
-                if (LIMITED) pos = pos < lim.cap ? total[e] + pos : -1;
-                if (pos >= 0) sorted_token[pos] = (int32_t)(a / k_max);
-                dest_pos[a] = pos;
-            } else if (a < n_flat) {
-                dest_pos[a] = -1;
-            }
-            __syncwarp();
-            if (e >= 0 && lane == __ffs(peers) - 1) r[e] += __popc(peers);
-            __syncwarp();
+        for (int w = 0; w < kDispWarps; ++w) {
+            const int32_t h = hist[w][e];
+            hist[w][e] = b;
+            b += h;
         }
     }
+    __syncthreads();
+
+    int32_t *run = hist[warp];
+    const unsigned lower = (1u << lane) - 1u;
+#pragma unroll
+    for (int j = 0; j < ITEMS; ++j) {
+        const int64_t a = base + (int64_t)j * 32 + lane;
+        const int e = eb[j];
+        const unsigned peers = pm[j];
+        if (e >= 0) {
+            int32_t pos = run[e] + __popc(peers & lower);
+            if (LIMITED) pos = pos < lim.cap ? total[e] + pos : -1;
+            if (pos >= 0) sorted_token[pos] = (int32_t)(a / k_max);
+            dest_pos[a] = pos;
+        } else if (a < n_flat) {
+            dest_pos[a] = -1;
+        }
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(peers) - 1) run[e] += __popc(peers);
+        __syncwarp();
+    }
     griddep_launch_dependents();
+}
+
+// Launches count + scatter for the segment size `items` picks.
+template <bool LIMITED>
+cudaError_t launch_dispatch(int items, int64_t S, cudaStream_t cs, const int32_t *ids,
+                            int64_t n_flat, int k_max, int E, int32_t *seg_total,
+                            int32_t *counts, int32_t *offsets, int32_t *sorted_token,
+                            int32_t *dest_pos, int32_t *d_status, Limits lim) {
+    const int Ep = seg_stride(E);
+    const dim3 grid((unsigned)S), block(kDispWarps * 32);
+    cudaError_t err;
+#define MOE_DISPATCH_CASE(IT)                                                                     \
+    case IT:                                                                                      \
+        err = launch_pdl(dispatch_count_kernel<IT>, grid, block, 0, cs, ids, n_flat, E, Ep,       \
+                         seg_total, d_status);                                                    \
+        if (err != cudaSuccess) return err;                                                       \
+        return launch_pdl(dispatch_scatter_kernel<IT, LIMITED>, grid, block, 0, cs, ids, n_flat,  \
+                          k_max, E, Ep, S, (const int32_t *)seg_total, counts, offsets,           \
+                          sorted_token, dest_pos, lim);
+    switch (items) {
+        MOE_DISPATCH_CASE(4)
+        MOE_DISPATCH_CASE(8)
+        MOE_DISPATCH_CASE(16)
+        default:
+            return cudaErrorInvalidValue;
+    }
+#undef MOE_DISPATCH_CASE
 }
 
 }  // namespace
@@ -269,7 +313,7 @@ extern "C" moe_status moe_dispatch_workspace_size(int64_t T, int32_t k_max, int3
     const int64_t n_flat = T * (int64_t)k_max;
     if (n_flat >= (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
     const int64_t S = num_segments(n_flat, warp_items(n_flat));
-    const size_t b = (size_t)S * (size_t)E * sizeof(int32_t) * (1 + kDispWarps);
+    const size_t b = (size_t)S * (size_t)seg_stride(E) * sizeof(int32_t);
     *bytes = (b + 255) / 256 * 256;
     return MOE_OK;
 }
@@ -292,18 +336,10 @@ extern "C" moe_status moe_dispatch(const int32_t *topk_ids, int64_t T, int32_t k
     const int items = warp_items(n_flat);
     const int64_t S = num_segments(n_flat, items);
     if (S > 0) {
-        int32_t *seg_total = static_cast<int32_t *>(workspace);
-        int32_t *warp_hist = seg_total + S * E;
-        if (launch_pdl(dispatch_count_kernel, dim3((unsigned)S), dim3(kDispWarps * 32), 0, cs,
-                       topk_ids, n_flat, (int)E, items, seg_total, warp_hist, d_status) !=
-            cudaSuccess) {
-            cudaGetLastError();
-            return MOE_ERR_CUDA;
-        }
-        if (launch_pdl(dispatch_scatter_kernel<false>, dim3((unsigned)S), dim3(kDispWarps * 32), 0,
-                       cs, topk_ids, n_flat, (int)k_max, (int)E, items, S,
-                       (const int32_t *)seg_total, (const int32_t *)warp_hist, counts, offsets,
-                       sorted_token, dest_pos, Limits{INT32_MAX, 1, nullptr}) != cudaSuccess) {
+        if (launch_dispatch<false>(items, S, cs, topk_ids, n_flat, (int)k_max, (int)E,
+                                   static_cast<int32_t *>(workspace), counts, offsets,
+                                   sorted_token, dest_pos, d_status,
+                                   Limits{INT32_MAX, 1, nullptr}) != cudaSuccess) {
             cudaGetLastError();
             return MOE_ERR_CUDA;
         }
@@ -359,19 +395,10 @@ extern "C" moe_status moe_dispatch_limited(const int32_t *topk_ids, int64_t T, i
     const int items = warp_items(n_flat);
     const int64_t S = num_segments(n_flat, items);
     if (S > 0) {
-        int32_t *seg_total = static_cast<int32_t *>(workspace);
-        int32_t *warp_hist = seg_total + S * E;
-        if (launch_pdl(dispatch_count_kernel, dim3((unsigned)S), dim3(kDispWarps * 32), 0, cs,
-                       topk_ids, n_flat, (int)E, items, seg_total, warp_hist, d_status) !=
-            cudaSuccess) {
-            cudaGetLastError();
-            return MOE_ERR_CUDA;
-        }
         const Limits lim{capacity > 0 ? capacity : INT32_MAX, pad, dropped};
-        if (launch_pdl(dispatch_scatter_kernel<true>, dim3((unsigned)S), dim3(kDispWarps * 32), 0,
-                       cs, topk_ids, n_flat, (int)k_max, (int)E, items, S,
-                       (const int32_t *)seg_total, (const int32_t *)warp_hist, counts, offsets,
-                       sorted_token, dest_pos, lim) != cudaSuccess) {
+        if (launch_dispatch<true>(items, S, cs, topk_ids, n_flat, (int)k_max, (int)E,
+                                  static_cast<int32_t *>(workspace), counts, offsets, sorted_token,
+                                  dest_pos, d_status, lim) != cudaSuccess) {
             cudaGetLastError();
             return MOE_ERR_CUDA;
         }
