@@ -232,7 +232,9 @@ def _dispatch(ids, E):
 @pytest.mark.parametrize("T,k,E,empty_frac,hot", [
     (1, 1, 1, 0.0, False), (1000, 8, 256, 0.0, False), (3001, 4, 128, 0.0, True),
     (777, 16, 128, 0.4, False), (5000, 6, 384, 0.0, False), (20000, 32, 512, 0.1, True),
-    (333, 3, 7, 0.2, False), (70000, 8, 256, 0.0, True)])
+    (333, 3, 7, 0.2, False), (70000, 8, 256, 0.0, True),
+    # 200 K slots: eight items a lane; E = 130: 33 quads of the segment-total rows
+    (25000, 8, 128, 0.3, True), (4000, 5, 130, 0.1, False)])
 def test_dispatch_parity(T, k, E, empty_frac, hot):
     g = _gen(T + k + E)
     ids = torch.randint(0, E, (T, k), generator=g, device=DEV, dtype=torch.int32)
