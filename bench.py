@@ -484,8 +484,8 @@ def run_ours(args):
             cur["s"] = s
             run_step(mark)
     else:
-        # The step captured once as a CUDA graph (no host launch overhead);
-        # stage boundaries are event-record nodes inside it, read after each replay.
+        # The step captured as CUDA graphs (no host launch overhead); event-record
+        # nodes inside them are read after each replay.
         gev = [torch.cuda.Event(enable_timing=True) for _ in range(nb)]
         for e in gev:
             e.record(stream)
