@@ -763,6 +763,142 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def ep_stage_bytes(T: int, d: int, k_max: int, n_assign: int, shared: bool) -> dict:
+    """Algorithmic bytes of the expert-parallel exchange kernels over all ranks:
+    layout reads ids and dest_pos and writes dest_rank and dest_row; permute
+    reads every token row once and writes each of its N copies; combine reads
+    the N expert rows (and the shared rows) and writes one row per token."""
+    slots = T * k_max
+    return {"ep_layout": 16 * slots,
+            "ep_permute": T * d * 2 + n_assign * d * 2 + 8 * slots,
+            "ep_combine": n_assign * d * 2 + T * d * 2 + (T * d * 2 if shared else 0) + 12 * slots}
+
+
+def run_ep_emulated(args):
+    """The expert-parallel exchange kernels with G ranks emulated on one GPU.
+
+    The workload's tokens are routed once, then split over G ranks.  Every
+    rank's buffers live on this device and the peer tables hold their
+    addresses, so each rank's moe_ep_permute stores into all G receive
+    buffers and its moe_ep_combine gathers from all G expert-output buffers,
+    exactly as over NVLink, but the rows cross HBM instead.  The ranks'
+    kernels run one after another on one stream (none waits on another)."""
+    import token_dispatch_moe_b200 as moe
+    from token_dispatch_moe_b200.ep import EpRank, recv_rows
+    from token_dispatch_moe_b200.path import RouterDispatch
+    from token_dispatch_moe_b200.workloads import WORKLOADS, make_inputs
+
+    G = args.ep_emulate
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    moe.load_library()
+    wl = WORKLOADS[args.workload]
+    if args.tokens:
+        wl = wl.scaled(args.tokens)
+    if wl.E % G or wl.T % G:
+        raise SystemExit(f"{wl.name}: E = {wl.E} and T = {wl.T} must split over {G} ranks")
+    inp = make_inputs(wl, device, with_y=False)
+    path = RouterDispatch(wl, device, fused=False)
+    logits = path.gate(inp["x"], inp["w"]) if wl.gate else inp["logits"]
+    path.route(logits, inp["bias"], inp["k_per_token"])
+    torch.cuda.synchronize()
+    Tr, k, d = wl.T // G, wl.k_max, wl.d
+    rows_of = lambda t, r: t[r * Tr:(r + 1) * Tr]  # noqa: E731
+    xs = [rows_of(inp["x"], r) for r in range(G)]
+    ids = [rows_of(path.topk_ids, r) for r in range(G)]
+    wts = [rows_of(path.topk_w, r) for r in range(G)]
+    sh = [rows_of(inp["shared"], r) if inp["shared"] is not None else None for r in range(G)]
+    ranks = [EpRank(Tr, k, wl.E, G, r, device) for r in range(G)]
+    for r in range(G):
+        ranks[r].dispatch(ids[r])
+    all_counts = torch.stack([rs.counts for rs in ranks])
+    rows = recv_rows(all_counts)
+    cap = max(max(rows), 1)
+    g = torch.Generator(device=device)
+    g.manual_seed(1000 * wl.index + 77)
+    recv = [torch.empty((cap, d), dtype=torch.bfloat16, device=device) for _ in range(G)]
+    ybuf = [torch.randn((cap, d), generator=g, device=device).to(torch.bfloat16) for _ in range(G)]
+    outs = [torch.empty((Tr, d), dtype=torch.bfloat16, device=device) for _ in range(G)]
+    recv_tab, y_tab = moe.peer_table(recv), moe.peer_table(ybuf)
+    stream = torch.cuda.current_stream(device)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=device)
+    names = ["ep_layout", "ep_permute", "ep_combine"]
+
+    def one(mark):
+        mark(0)
+        for r in range(G):
+            ranks[r].layout(all_counts, ids[r])
+        mark(1)
+        for r in range(G):
+            ranks[r].permute(xs[r], recv_tab, cap)
+        mark(2)
+        for r in range(G):
+            ranks[r].combine(y_tab, wts[r], sh[r], outs[r], cap)
+        mark(3)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        one(lambda i: None)
+    torch.cuda.synchronize()
+    bad = [r for r in range(G) if ranks[r].status.item() != 0]
+    if bad:
+        raise RuntimeError(f"device status on ranks {bad}: "
+                           f"{moe.moe_status_string(ranks[bad[0]].status.item())}")
+    # The 3 x G launches captured as one CUDA graph, so that host launch time
+    # does not open gaps between the short kernels; event-record nodes at the
+    # stage boundaries are read after each replay.
+    gev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for e in gev:
+        e.record(stream)
+    torch.cuda.synchronize()
+    cudart = ctypes.CDLL("libcudart.so.12")
+    cudart.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
+    cap_stream = torch.cuda.Stream(device)
+
+    def mark(i):
+        if cudart.cudaEventRecordWithFlags(gev[i].cuda_event, cap_stream.cuda_stream, 1) != 0:
+            raise RuntimeError("cudaEventRecordWithFlags failed")
+
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=cap_stream, capture_error_mode="relaxed"):
+        one(mark)
+    graph.replay()
+    torch.cuda.synchronize()
+    times = {n: [] for n in names}
+    with ClockSampler(device.index) as clk:
+        t_warm = time.perf_counter()
+        while time.perf_counter() - t_warm < 0.3:  # let the sampler start under load (untimed)
+            graph.replay()
+            torch.cuda.synchronize()
+        for _ in range(args.steps):
+            flush.zero_()  # L2 flush before every timed pass, outside its events
+            graph.replay()
+            torch.cuda.synchronize()
+            for i, n in enumerate(names):
+                times[n].append(gev[i].elapsed_time(gev[i + 1]))
+    n_assign = int(sum(rows))
+    nbytes = ep_stage_bytes(wl.T, d, k, n_assign, inp["shared"] is not None)
+    hbm, _, _, peak_kind = load_peaks()
+    stages = {}
+    for n in names:
+        ms = statistics.fmean(times[n])
+        gbs = nbytes[n] / (ms / 1e3) / 1e9
+        stages[n] = {"us": round(ms * 1e3, 2), "bytes": nbytes[n], "GB_s": round(gbs, 1),
+                     "frac_hbm": round(gbs / hbm, 4)}
+    print(json.dumps({
+        "metric": "expert-parallel exchange kernels, ranks emulated on one GPU",
+        "unit": "GB/s per kernel", "ranks": G, "steps": args.steps, "warmup": args.warmup,
+        "launch": "CUDA graph of the G ranks' launches, one stage after another",
+        "config": {"workload": wl.name, "tokens_per_rank": Tr, "hidden": d, "experts": wl.E,
+                   "experts_per_rank": wl.E // G, "rows_sent": n_assign,
+                   "recv_rows_per_rank": rows,
+                   "l2": f"flushed before every timed pass ({flush.numel() * 4 >> 20} MiB write)",
+                   "links": "none: every buffer is on this GPU, so rows cross HBM, not NVLink"},
+        "stages": stages, "peak": {"hbm_gbs": hbm, "source": peak_kind},
+        "clocks": clk.summary()}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -789,7 +925,13 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0,
                     help="seconds of single-core oracle work for the CPU baseline")
+    ap.add_argument("--ep-emulate", type=int, default=0, metavar="G",
+                    help="time the expert-parallel exchange kernels with G ranks emulated on "
+                         "this one GPU (a separate measurement, not the chain)")
     args = ap.parse_args(argv)
+    if args.ep_emulate:
+        run_ep_emulated(args)
+        return
     world, _, _ = dist_env()
     if world != args.gpus and not (world == 1 and args.gpus == 1):
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)

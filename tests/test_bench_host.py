@@ -34,6 +34,23 @@ def test_stage_bytes_qwen3(bench):
     assert f["gate_route"] == T * d * 2 + E * d * 2 + T * k * 8 + T * 4
 
 
+def test_ep_stage_bytes_match_the_local_kernels(bench):
+    """The exchange moves the same rows as permute and combine; its only extra
+    bytes are the second routing table (dest_rank beside dest_row)."""
+    wl = WORKLOADS["qwen3_dynk"]
+    T, d, k = wl.T, wl.d, wl.k_max
+    n = 150000
+    local = bench.stage_bytes(wl, n, fused=False)
+    ep = bench.ep_stage_bytes(T, d, k, n, shared=False)
+    assert ep["ep_permute"] - local["permute"] == 4 * T * k
+    assert ep["ep_combine"] - local["combine"] == 4 * T * k
+    assert ep["ep_layout"] == 16 * T * k
+    v3 = WORKLOADS["deepseek_v3"]
+    with_shared = bench.ep_stage_bytes(v3.T, v3.d, v3.k_max, n, shared=True)
+    without = bench.ep_stage_bytes(v3.T, v3.d, v3.k_max, n, shared=False)
+    assert with_shared["ep_combine"] - without["ep_combine"] == v3.T * v3.d * 2
+
+
 def test_stage_bytes_capacity(bench):
     wl = WORKLOADS["llama4_top1_capacity"]
     T, d, E = wl.T, wl.d, wl.E

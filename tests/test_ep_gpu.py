@@ -56,7 +56,8 @@ def _emulated_exchange(G, T, k, E, d, seed, hot=False, cap_extra=0):
 @pytest.mark.parametrize("G,T,k,E,d,hot", [(1, 300, 4, 8, 64, False), (2, 500, 2, 8, 128, False),
                                            (4, 1000, 8, 64, 256, True),
                                            (8, 777, 6, 256, 7168, False),
-                                           (8, 64, 1, 8, 2048, True)])
+                                           (8, 64, 1, 8, 2048, True),
+                                           (2, 300, 3, 16, 768, False)])  # two vectors a lane
 def test_ep_exchange_parity(G, T, k, E, d, hot):
     xs, ids, ws, sh, ranks, all_counts, rows, cap, recv = _emulated_exchange(
         G, T, k, E, d, 77 + G * 13 + T, hot)
