@@ -119,6 +119,7 @@ __global__ void __launch_bounds__(kDispWarps * 32)
     griddep_wait();
 
     // This warp's ids: loaded once, kept in registers for both passes below.
+    // An id outside [-1, E) counts as empty here; the count kernel reported it.
     const int64_t base = (s * kDispWarps + warp) * (int64_t)ITEMS * 32;
     bool bad = false;
     int eb[ITEMS];
