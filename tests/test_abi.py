@@ -47,12 +47,25 @@ def test_status_strings(lib):
     assert "timed out" in moe.moe_status_string(moe.MOE_ERR_TIMEOUT)
 
 
+def _expected_workspace(T, k, E):
+    """One int32 per (segment, expert), the expert row padded to whole 16-byte
+    quads; a segment is 8 warps x 32 lanes x `items` slots, items the smallest
+    of 4, 8, 16 for which 148 segments cover every slot; rounded up to 256 B."""
+    n = T * k
+    items = 4
+    while items * 32 * 8 * 148 < n and items < 16:
+        items *= 2
+    segs = -(-n // (items * 32 * 8))
+    b = segs * (-(-E // 4) * 4) * 4
+    return -(-b // 256) * 256
+
+
 def test_workspace_size(lib):
-    # one int32 per (segment, expert); segments of 32 * items slots, rounded to 256 B
     assert moe.moe_dispatch_workspace_size(0, 8, 256) == 0
-    b = moe.moe_dispatch_workspace_size(16384, 16, 128)
-    n_flat = 16384 * 16
-    assert b >= (n_flat // (32 * 64)) * 128 * 4 and b % 256 == 0
+    for T, k, E in [(16384, 16, 128), (4000, 5, 130), (65536, 32, 512), (1, 1, 1),
+                    (70000, 8, 256), (25000, 8, 7)]:
+        assert moe.moe_dispatch_workspace_size(T, k, E) == _expected_workspace(T, k, E)
+    assert moe.moe_dispatch_workspace_size(16384, 16, 128) == 128 * 128 * 4  # 128 segments of 8 items
     assert moe.moe_dispatch_workspace_size(1, 1, 1) == 256
     with pytest.raises(moe.MoeError):
         moe.moe_dispatch_workspace_size(10, 33, 8)   # k_max > 32
