@@ -789,14 +789,14 @@ def run_ep_emulated(args):
     from token_dispatch_moe_b200.workloads import WORKLOADS, make_inputs
 
     G = args.ep_emulate
-    device = torch.device("cuda", 0)
-    torch.cuda.set_device(device)
-    moe.load_library()
     wl = WORKLOADS[args.workload]
     if args.tokens:
         wl = wl.scaled(args.tokens)
-    if wl.E % G or wl.T % G:
+    if G < 1 or wl.E % G or wl.T % G:
         raise SystemExit(f"{wl.name}: E = {wl.E} and T = {wl.T} must split over {G} ranks")
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    moe.load_library()
     inp = make_inputs(wl, device, with_y=False)
     path = RouterDispatch(wl, device, fused=False)
     logits = path.gate(inp["x"], inp["w"]) if wl.gate else inp["logits"]

@@ -51,6 +51,16 @@ def test_ep_stage_bytes_match_the_local_kernels(bench):
     assert with_shared["ep_combine"] - without["ep_combine"] == v3.T * v3.d * 2
 
 
+def test_ep_emulate_refuses_uneven_splits(bench):
+    """Checked before any device work: mixtral_tiny's 8 experts do not split
+    over 3 ranks, and 16384 tokens do not split over 3 either."""
+    for argv in (["--ep-emulate", "3", "--workload", "mixtral_tiny"],
+                 ["--ep-emulate", "3"]):
+        with pytest.raises(SystemExit) as err:
+            bench.main(argv)
+        assert "must split over 3 ranks" in str(err.value)
+
+
 def test_stage_bytes_capacity(bench):
     wl = WORKLOADS["llama4_top1_capacity"]
     T, d, E = wl.T, wl.d, wl.E
