@@ -44,7 +44,7 @@ def _worker(rank, world, port, out):
 
 def test_count_exchange_and_receive_sizes():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()  # no fork of a threaded process
     out = mgr.dict()
     mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     (c0, r0), (c1, r1) = out[0], out[1]

@@ -34,7 +34,7 @@ def _worker(rank, world, port, out):
 
 def test_two_rank_max_and_throughput():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()  # no fork of a threaded process
     out = mgr.dict()
     mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     (m0, v0, s0), (m1, v1, s1) = out[0], out[1]
