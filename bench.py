@@ -318,32 +318,49 @@ def oracle_inputs(wl, inp: dict, n_tokens: int, experts=None) -> dict:
     return h
 
 
-def oracle_chain(wl, h: dict, hash_layer: bool = False) -> None:
+def oracle_chain(wl, h: dict, hash_layer: bool = False, stage_s: dict | None = None) -> None:
     """The path computed by the fp64 CPU oracle (single thread): gate, route,
     dispatch, permute, [the experts' FFN when h holds their weights], combine,
     on the sample held in h; or the hash-routed layer's chain (gate, hash
-    route, dispatch, permute)."""
+    route, dispatch, permute).  stage_s, if given, receives each stage's wall
+    seconds."""
     import oracle
+    t_last = [time.perf_counter()]
+
+    def lap(name):
+        now = time.perf_counter()
+        if stage_s is not None:
+            stage_s[name] = stage_s.get(name, 0.0) + now - t_last[0]
+        t_last[0] = now
+
     score = {"softmax": oracle.SOFTMAX, "sigmoid": oracle.SIGMOID,
              "sqrt_softplus": oracle.SQRT_SOFTPLUS, "topk_softmax": oracle.TOPK_SOFTMAX}[wl.score]
     logits = oracle.gate_rows(h["x"], h["w"]).astype(np.float32) if wl.gate else h["logits"]
+    if wl.gate:
+        lap("gate_gemm")
     if hash_layer:
         r = oracle.hash_route(h["token_ids"], h["tid2eid"], num_experts=wl.E, logits=logits,
                               score=score, renormalize=wl.renormalize,
                               route_scale=wl.route_scale)
+        lap("hash_route")
         dsp = oracle.dispatch(r["ids"], wl.E)
+        lap("dispatch")
         oracle.permute(h["x"], dsp["dest_pos"], int(dsp["offsets"][-1]))
+        lap("permute")
         return
     r = oracle.route(logits, k_max=wl.k_max, score=score, bias=h["bias"], k_per_token=h["kpt"],
                      n_groups=wl.n_groups, topk_groups=wl.topk_groups, group_topn=wl.group_topn,
                      renormalize=wl.renormalize, route_scale=wl.route_scale)
+    lap("route")
     if wl.limited:  # the same capacity rule, applied to the sample's own tokens
         dsp = oracle.dispatch_limited(r["ids"], wl.E, capacity=wl.scaled(h["T"]).capacity,
                                       pad=wl.pad)
     else:
         dsp = oracle.dispatch(r["ids"], wl.E)
+    lap("dispatch")
     n = int(dsp["offsets"][-1])
     xs = oracle.permute(h["x"], dsp["dest_pos"], n)
+    lap("permute")
     y = h["y"]
     if h.get("experts") is not None:
         ex = h["experts"]
@@ -353,12 +370,15 @@ def oracle_chain(wl, h: dict, hash_layer: bool = False) -> None:
         hv = oracle.expert_gate_up(xs, dsp["offsets"], ex["w1"], ex["w3"], rows, act=act,
                                    b1=ex["b1"], b3=ex["b3"])
         hid[rows] = torch.from_numpy(hv).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        lap("expert_gate_up")
         yv = oracle.expert_down(hid, dsp["offsets"], ex["w2"], rows, b2=ex["b2"])
         y = np.zeros((max(n, 1), wl.d), np.uint16)
         y[rows] = torch.from_numpy(yv).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        lap("expert_down")
     if wl.combine:
         oracle.combine(y[:max(n, 1)], r["w"].astype(np.float32), dsp["dest_pos"],
                        h["shared"], want_mag=False)
+        lap("combine")
 
 
 def oracle_sample_size(wl, inp, budget_s: float, experts=None, hash_layer=False) -> int:
@@ -714,12 +734,14 @@ def measure_e2e(wl, inp, path, device, stream, steps, world, experts=None, hash_
 def cpu_baseline(wl, inp, budget_s: float, experts=None, hash_layer=False) -> dict:
     n = oracle_sample_size(wl, inp, budget_s, experts, hash_layer)
     h = oracle_inputs(wl, inp, n, experts)
+    stage_s = {}
     t0 = time.perf_counter()
-    oracle_chain(wl, h, hash_layer)
+    oracle_chain(wl, h, hash_layer, stage_s)
     dt = time.perf_counter() - t0
     return {"value": round(n / dt, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"first {n} of {wl.T} tokens of {wl.name}, full chain in fp64, "
-                      f"{dt:.1f} s on one host core"}
+                      f"{dt:.1f} s on one host core",
+            "stage_s": {k: round(v, 3) for k, v in stage_s.items()}}
 
 
 # ---------------------------------------------------------- reference arm
@@ -742,9 +764,10 @@ def run_reference(args):
     h = oracle_inputs(wl, inp, per_step, experts)
     for _ in range(args.warmup):
         oracle_chain(wl, h, hl)
+    stage_s = {}
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_chain(wl, h, hl)
+        oracle_chain(wl, h, hl, stage_s)
     dt = time.perf_counter() - t0
     value = per_step * args.steps / dt
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
@@ -757,7 +780,9 @@ def run_reference(args):
                        "parallelism": "single host core"},
             "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": 1,
                              "kind": "oracle",
-                             "sample": f"first {per_step} of {wl.T} tokens per step"},
+                             "sample": f"first {per_step} of {wl.T} tokens per step",
+                             "stage_ms_per_step": {k: round(v / args.steps * 1e3, 3)
+                                                   for k, v in stage_s.items()}},
             "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

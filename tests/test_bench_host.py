@@ -87,7 +87,11 @@ def test_oracle_chain_runs_on_cpu_inputs(bench, name):
     assert h["T"] == 40 and h["x"].shape == (40, wl.d)
     n = int(h["kpt"].sum()) if wl.k_choices else 40 * wl.k_max
     assert h["y"].shape[0] >= n
-    bench.oracle_chain(wl, h)
+    stage_s = {}
+    bench.oracle_chain(wl, h, stage_s=stage_s)
+    # the oracle's per-stage wall times carry the GPU stages' names
+    assert set(stage_s) == set(bench.stage_bytes(wl, n))
+    assert all(v >= 0.0 for v in stage_s.values())
     assert bench.oracle_sample_size(wl, inp, 0.05) >= 8
     if wl.k_choices:
         assert set(np.unique(h["kpt"])) <= set(wl.k_choices)
