@@ -338,6 +338,71 @@ def pin_dynamic_k_prefix():
         assert np.array_equal(dyn["w"][t, :k], full["w"][t, :k])
 
 
+def pin_weights_for_ids():
+    """Weights of a selection made elsewhere ("DeepSeek-V3.2-Exp - Select
+    experts", gate forward: gather the unbiased scores of the chosen experts,
+    divide by their sum, times route_scale; "Crate ferrox_moe",
+    route_top_k_softmax_weight: softmax over the chosen logits).
+
+    (1) Against Python's math module (bf_weights) on arbitrary id lists: slots
+        in any order, -1 holes anywhere, all four scores, with and without
+        renormalisation, several route_scales.
+    (2) On the router's own selections (bias, groups, per-token k), the weights
+        of the chosen ids are the router's weights, bit for bit: the bias only
+        selects, it never weighs.
+    (3) An id >= E is refused."""
+    rng = np.random.default_rng(21)
+    for score in (oracle.SOFTMAX, oracle.SIGMOID, oracle.SQRT_SOFTPLUS, oracle.TOPK_SOFTMAX):
+        for renorm, scale in ((True, 2.5), (False, 1.0), (True, 1.0), (False, 0.75)):
+            T, E, k_max = 40, 13, 5
+            lg = (rng.normal(size=(T, E)) * 2.0).astype(np.float32)
+            ids = np.full((T, k_max), -1, np.int32)
+            for t in range(T):
+                n = int(rng.integers(0, k_max + 1))
+                chosen = rng.permutation(E)[:n]            # any experts, any order
+                slots = np.sort(rng.permutation(k_max)[:n])  # holes anywhere
+                ids[t, slots] = chosen
+            w = oracle.weights_for_ids(lg, ids, score=score, renormalize=renorm,
+                                       route_scale=scale)
+            for t in range(T):
+                l = [float(v) for v in lg[t]]
+                s = bf_scores(l, score)
+                live = [j for j in range(k_max) if ids[t, j] >= 0]
+                want = bf_weights(l, s, [int(ids[t, j]) for j in live], score, renorm, scale)
+                exp = np.zeros(k_max)
+                exp[live] = want
+                assert _rel_close(w[t], exp, 1e-12, 1e-300), (score, renorm, t, w[t], exp)
+    # (2) the router's selections, weighed again
+    T, E = 96, 64
+    lg = rng.normal(size=(T, E)).astype(np.float32)
+    b = rng.uniform(-0.1, 0.1, size=E).astype(np.float32)
+    kpt = rng.choice([0, 1, 3, 6, 8], size=T).astype(np.int32)
+    for score in (oracle.SOFTMAX, oracle.SIGMOID, oracle.SQRT_SOFTPLUS, oracle.TOPK_SOFTMAX):
+        for bias, G, TG, topn, kp, renorm, scale in (
+                (b, 8, 4, 2, None, True, 2.5), (None, 1, 1, 1, kpt, True, 1.0),
+                (b, 4, 2, 2, kpt, False, 1.0), (None, 8, 3, 1, None, False, 1.5)):
+            r = oracle.route(lg, k_max=8, score=score, bias=bias, k_per_token=kp, n_groups=G,
+                             topk_groups=TG, group_topn=topn, renormalize=renorm,
+                             route_scale=scale)
+            w = oracle.weights_for_ids(lg, r["ids"], score=score, renormalize=renorm,
+                                       route_scale=scale)
+            assert np.array_equal(w, r["w"]), (score, G, renorm)
+            # a permutation of the slots permutes the weights and nothing else
+            perm = rng.permutation(8)
+            wp = oracle.weights_for_ids(lg, r["ids"][:, perm], score=score, renormalize=renorm,
+                                        route_scale=scale)
+            assert _rel_close(wp, r["w"][:, perm], 1e-13, 1e-300), (score, G, renorm)
+    # (3) an id past the last expert
+    import ctypes
+    bad = np.array([[0, 3]], np.int32)
+    lg1 = np.zeros((1, 3), np.float32)
+    out = np.empty((1, 2), np.float64)
+    st = oracle._load().oracle_weights_for_ids(lg1.ctypes.data, bad.ctypes.data, 1, 3, 2,
+                                              oracle.SOFTMAX, 1, ctypes.c_double(1.0),
+                                              out.ctypes.data)
+    assert st == oracle.ERR_INDEX, st
+
+
 def pin_status_and_nan():
     lg = np.array([[0.5, np.nan, 2.0, -1.0]], np.float32)
     r = oracle.route(lg, k_max=3, score=oracle.SIGMOID, renormalize=False)
@@ -633,8 +698,8 @@ def pin_combine_cases():
 PINS = [pin_score_closed_forms, pin_score_library_cases, pin_status_and_nan,
         pin_gate_integer_exact, pin_gate_torch_fp64, pin_hash_lookup, pin_dispatch_library,
         pin_dispatch_limited, pin_ep_layout, pin_route_grouped, pin_expert_ffn,
-        pin_permute_copy, pin_combine_cases, pin_weight_invariants, pin_dynamic_k_prefix,
-        pin_deepseek_worked_cases, pin_brute_force_selection]
+        pin_permute_copy, pin_combine_cases, pin_weight_invariants, pin_weights_for_ids,
+        pin_dynamic_k_prefix, pin_deepseek_worked_cases, pin_brute_force_selection]
 
 
 def run_all(stop_at_first: bool = True) -> list[str]:

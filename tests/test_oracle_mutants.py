@@ -33,6 +33,13 @@ MUTANTS = {
     "group_keep_one_less": ("for (int32_t i = 0; i < topk_groups; ++i) kept[grp[i].id] = 1;",
                             "for (int32_t i = 0; i + 1 < topk_groups; ++i) kept[grp[i].id] = 1;"),
     "no_renormalise": ("    if (renormalize) {\n        double sum", "    if (0) {\n        double sum"),
+    "weights_for_ids_row_offset": (
+        "        row_scores(logits + t * E, E, score, s);\n        row_weights(logits + t * E, s, ids + t * k_max,",
+        "        row_scores(logits + t * k_max, E, score, s);\n        row_weights(logits + t * E, s, ids + t * k_max,"),
+    "weights_for_ids_ids_row": ("row_weights(logits + t * E, s, ids + t * k_max, k_max,",
+                                "row_weights(logits + t * E, s, ids + t, k_max,"),
+    "weights_for_ids_no_renormalise": ("ids + t * k_max, k_max, score, renormalize, route_scale,",
+                                       "ids + t * k_max, k_max, score, 0, route_scale,"),
     "route_scale_ignored": ("if (ids[j] >= 0) w[j] *= route_scale;", "if (ids[j] >= 0) w[j] *= 1.0;"),
     "gptoss_softmax_all": ("    if (score == ORACLE_TOPK_SOFTMAX) {\n        double m",
                            "    if (0) {\n        double m"),
