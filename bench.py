@@ -43,7 +43,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
-DEFAULT_WORKLOAD = "qwen3_dynk"
+DEFAULT_WORKLOAD = "deepseek_v3"
 METRIC = "routed tokens/s (gate->top-k->permute->combine); % of HBM/tensor roofline"
 
 
@@ -670,7 +670,10 @@ def measure_e2e(wl, inp, path, device, stream, steps, world, experts=None, hash_
     keys = ("x", "w", "token_ids") if hash_layer else \
         ("x", "w", "logits", "bias", "k_per_token", "y", "shared")
     names = [k for k in keys if inp[k] is not None]
-    host = {k: inp[k].cpu().pin_memory() for k in names}
+    # pinned host copies, made without a pageable intermediate (deepseek_v3's
+    # x, y and shared rows are 9.4 GB)
+    host = {k: torch.empty(inp[k].shape, dtype=inp[k].dtype, pin_memory=True).copy_(inp[k])
+            for k in names}
     paths = [path, make_path() if make_path is not None else path]
     devs = [{k: torch.empty_like(inp[k]) for k in names} for _ in range(2)]
     fulls = []

@@ -267,9 +267,12 @@ moe_status moe_dispatch_limited(const int32_t *topk_ids, int64_t T, int32_t k_ma
  * moe_dispatch_workspace_size() exceeds 4 MiB are rejected with
  * MOE_ERR_UNSUPPORTED and nothing is launched.  The library allocates and frees
  * nothing here either.
- * The first call on a device (made with that device current) looks up the
- * scratch array's device address; make that first call before any stream
- * capture.  All calls share the one array: two calls whose work overlaps on
+ * The scratch array's device address is looked up (cudaGetSymbolAddress) by
+ * the first call in each CUDA context and cached under that context's unique
+ * id, so a context destroyed and created again (e.g. after cudaDeviceReset) is
+ * looked up afresh; that first call may create the device's primary context,
+ * so make it before any stream capture.  Each device's context has its own
+ * copy of the array.  All calls share the one array: two calls whose work overlaps on
  * the GPU (different streams, or different host threads) race and give wrong
  * results; serialise them.  The array keeps the last call's contents, but no
  * call depends on them: everything a call reads from it, it wrote first.

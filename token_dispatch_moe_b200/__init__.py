@@ -121,7 +121,14 @@ def _ptr(t):
 
 
 def _stream(stream):
+    """Raw handle of the stream to launch on (torch's current stream if None).
+    A torch stream of another device than the current one is refused: the
+    library launches on the current device, with its kernels reading the
+    tensors' addresses there."""
     s = torch.cuda.current_stream() if stream is None else stream
+    if hasattr(s, "device") and s.device.index != torch.cuda.current_device():
+        raise ValueError(f"stream is on {s.device}, the current device is "
+                         f"cuda:{torch.cuda.current_device()}")
     return s.cuda_stream if hasattr(s, "cuda_stream") else s
 
 
@@ -137,6 +144,9 @@ def _need(t, dtype, name, ndim=None):
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}, the current device is "
+                         f"cuda:{torch.cuda.current_device()}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if ndim is not None and t.dim() != ndim:

@@ -23,7 +23,9 @@
 //               same id (popcount of lower lanes in the match mask), writing
 //               sorted_token and dest_pos.
 // Workspace: seg_total [S][Ep] int32, Ep = E rounded up to a multiple of 4.
-#include <atomic>
+#include <cuda.h>
+
+#include <mutex>
 
 #include "common.cuh"
 
@@ -419,17 +421,88 @@ extern "C" moe_status moe_dispatch_limited(const int32_t *topk_ids, int64_t T, i
 // themselves.  Its scratch is this file-scope device array: every GPU that
 // loads the library holds these 4 MiB until the process exits.  Host code must
 // not pass the array's name to a kernel (on the host it is only a stand-in);
-// the device address is fetched with cudaGetSymbolAddress once per device and
-// cached.
+// the device address is fetched with cudaGetSymbolAddress in the calling
+// thread's current context and cached under that context's unique id, so a
+// context that is destroyed and created again (cudaDeviceReset, a primary
+// context released and retained again) is looked up afresh instead of reusing
+// an address of the old one.
 namespace moe {
 namespace {
 constexpr size_t kStaticScratchBytes = size_t(4) << 20;
-constexpr int kMaxDevices = 64;
-std::atomic<void *> g_static_scratch_addr[kMaxDevices];
+constexpr int kScratchCacheSlots = 64;
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+template <typename Fn>
+Fn driver_fn(const char *name) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return reinterpret_cast<Fn>(p);
+}
+
+// Unique id (for the life of the process) of the calling thread's current
+// context; false when no context is current or the driver cannot tell.
+bool current_context_id(unsigned long long &id) {
+    static const CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    CUcontext ctx = nullptr;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+    return get_id(ctx, &id) == CUDA_SUCCESS;
+}
+
+// (context id -> scratch address) of the contexts seen so far; a full table
+// overwrites its oldest entry.  Context ids are never reused, so an entry of a
+// destroyed context can only go unused, never match a new one.
+struct ScratchCache {
+    std::mutex mu;
+    unsigned long long ctx[kScratchCacheSlots] = {};
+    void *addr[kScratchCacheSlots] = {};
+    int next = 0;
+};
+ScratchCache g_scratch_cache;
 }  // namespace
 }  // namespace moe
 
 static __device__ __align__(256) int32_t g_dispatch_scratch[moe::kStaticScratchBytes / sizeof(int32_t)];
+
+namespace moe {
+namespace {
+// Device address of g_dispatch_scratch in the current context (looked up on
+// the first call in each context, with cudaGetSymbolAddress; that lookup may
+// create the device's primary context, so it must not run inside a stream
+// capture), or nullptr on a CUDA error.
+void *static_scratch() {
+    unsigned long long id = 0;
+    bool have_id = current_context_id(id);
+    if (have_id) {
+        std::lock_guard<std::mutex> lock(g_scratch_cache.mu);
+        for (int i = 0; i < kScratchCacheSlots; ++i)
+            if (g_scratch_cache.ctx[i] == id && g_scratch_cache.addr[i]) return g_scratch_cache.addr[i];
+    }
+    void *addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_dispatch_scratch) != cudaSuccess || !addr) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    // The lookup makes the device's primary context current if none was.
+    if (!have_id) have_id = current_context_id(id);
+    if (have_id) {
+        std::lock_guard<std::mutex> lock(g_scratch_cache.mu);
+        const int i = g_scratch_cache.next;
+        g_scratch_cache.ctx[i] = id;
+        g_scratch_cache.addr[i] = addr;
+        g_scratch_cache.next = (i + 1) % kScratchCacheSlots;
+    }
+    return addr;
+}
+}  // namespace
+}  // namespace moe
 
 extern "C" moe_status moe_dispatch_static(const int32_t *topk_ids, int64_t T, int32_t k_max,
                                           int32_t E, int32_t *counts, int32_t *offsets,
@@ -440,22 +513,8 @@ extern "C" moe_status moe_dispatch_static(const int32_t *topk_ids, int64_t T, in
     moe_status st = moe_dispatch_workspace_size(T, k_max, E, &need);
     if (st != MOE_OK) return st;
     if (need > kStaticScratchBytes) return MOE_ERR_UNSUPPORTED;  // beyond the fixed scratch
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) {
-        cudaGetLastError();
-        return MOE_ERR_CUDA;
-    }
-    if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
-    void *addr = g_static_scratch_addr[dev].load(std::memory_order_acquire);
-    if (!addr) {
-        // First call on this device (with it current): resolve the array's
-        // device address.  Two threads racing here store the same value.
-        if (cudaGetSymbolAddress(&addr, g_dispatch_scratch) != cudaSuccess || !addr) {
-            cudaGetLastError();
-            return MOE_ERR_CUDA;
-        }
-        g_static_scratch_addr[dev].store(addr, std::memory_order_release);
-    }
+    void *addr = static_scratch();
+    if (!addr) return MOE_ERR_CUDA;
     // Every scratch entry a dispatch reads is written earlier by the same
     // dispatch, so the array needs no clearing between calls.
     return moe_dispatch(topk_ids, T, k_max, E, counts, offsets, sorted_token, dest_pos, addr,
