@@ -22,6 +22,8 @@
  *   moe_ep_layout / moe_ep_permute / moe_ep_combine
  *                             expert-parallel exchange over peer memory
  *   moe_dispatch_static       dispatch without a caller workspace
+ *   moe_permute_bounded / moe_combine_bounded
+ *                             permute / combine with dest_pos bounds-checked
  *   moe_wait_probe            diagnostic for the bounded-wait timeout path
  *
  * Conventions shared by every entry point:
@@ -305,6 +307,29 @@ moe_status moe_permute(const moe_bf16_t *x, const int32_t *dest_pos, int64_t T, 
 moe_status moe_combine(const moe_bf16_t *y, const float *topk_w, const int32_t *dest_pos,
                        const moe_bf16_t *shared, int64_t T, int32_t k_max, int32_t d,
                        moe_bf16_t *out, moe_stream_t stream);
+
+/*
+ * moe_permute_bounded / moe_combine_bounded -- moe_permute and moe_combine
+ * with every dest_pos checked against the rows the caller's buffer holds
+ * (xs_rows for permute, y_rows for combine): a value outside [-1, rows) is
+ * skipped (no row is read or written for that slot) and reported in
+ * *d_status (nullable) as MOE_ERR_DEVICE_INDEX.  Otherwise the same
+ * arguments, results and limits as the plain calls.  The plain calls trust
+ * dest_pos as moe_dispatch wrote it; in a library built with MOE_CHECKED
+ * they check it as well, against T * k_max rows (the most a dispatch of T
+ * tokens fills; use these bounded calls for padded layouts, whose
+ * moe_dispatch_limited_rows can exceed that), and skip without reporting,
+ * having no status argument.  (The pages' combine, "Crate ferrox_moe",
+ * combine_expert_outputs, has no index to check: these exist for callers
+ * that pass dest_pos from elsewhere.)
+ */
+moe_status moe_permute_bounded(const moe_bf16_t *x, const int32_t *dest_pos, int64_t T,
+                               int32_t k_max, int32_t d, moe_bf16_t *xs, int64_t xs_rows,
+                               int32_t *d_status, moe_stream_t stream);
+moe_status moe_combine_bounded(const moe_bf16_t *y, const float *topk_w, const int32_t *dest_pos,
+                               const moe_bf16_t *shared, int64_t T, int32_t k_max, int32_t d,
+                               int64_t y_rows, moe_bf16_t *out, int32_t *d_status,
+                               moe_stream_t stream);
 
 /*
  * moe_wait_probe -- diagnostic (no counterpart in the pages): one warp runs the

@@ -24,7 +24,7 @@ __all__ = [
     "MOE_ERR_DEVICE_INDEX", "MOE_ERR_TIMEOUT", "MOE_ERR_NAN_LOGIT",
     "moe_status_string", "moe_gate_gemm", "moe_gate_route", "moe_route", "moe_hash_route",
     "moe_dispatch_workspace_size", "moe_dispatch", "moe_dispatch_static", "moe_permute",
-    "moe_combine",
+    "moe_combine", "moe_permute_bounded", "moe_combine_bounded",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -99,6 +99,8 @@ def load_library(path: str | None = None):
                                   ctypes.c_size_t, P, P], st),
         "moe_permute": ([P, P, i64, i32, i32, P, P], st),
         "moe_combine": ([P, P, P, P, i64, i32, i32, P, P], st),
+        "moe_permute_bounded": ([P, P, i64, i32, i32, P, i64, P, P], st),
+        "moe_combine_bounded": ([P, P, P, P, i64, i32, i32, i64, P, P, P], st),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -455,3 +457,37 @@ def moe_combine(y, topk_w, dest_pos, shared, out, stream=None):
         raise ValueError("shape mismatch")
     _check(load_library().moe_combine(_ptr(y), _ptr(topk_w), _ptr(dest_pos), _ptr(shared), T,
                                       k_max, d, _ptr(out), _stream(stream)), "moe_combine")
+
+
+def moe_permute_bounded(x, dest_pos, xs, d_status=None, stream=None):
+    """moe_permute with every dest_pos checked against xs's rows: a value
+    outside [-1, xs rows) is skipped and reported in d_status."""
+    _need(x, torch.bfloat16, "x", 2)
+    _need(dest_pos, torch.int32, "dest_pos", 2)
+    _need(xs, torch.bfloat16, "xs", 2)
+    _need(d_status, torch.int32, "d_status")
+    T, d = x.shape
+    if dest_pos.shape[0] != T or xs.shape[1] != d:
+        raise ValueError("shape mismatch")
+    _check(load_library().moe_permute_bounded(_ptr(x), _ptr(dest_pos), T, dest_pos.shape[1], d,
+                                              _ptr(xs), xs.shape[0], _ptr(d_status),
+                                              _stream(stream)), "moe_permute_bounded")
+
+
+def moe_combine_bounded(y, topk_w, dest_pos, shared, out, d_status=None, stream=None):
+    """moe_combine with every dest_pos checked against y's rows: a value
+    outside [-1, y rows) is skipped (its term left out) and reported."""
+    _need(y, torch.bfloat16, "y", 2)
+    _need(topk_w, torch.float32, "topk_w", 2)
+    _need(dest_pos, torch.int32, "dest_pos", 2)
+    _need(shared, torch.bfloat16, "shared", 2)
+    _need(out, torch.bfloat16, "out", 2)
+    _need(d_status, torch.int32, "d_status")
+    T, d = out.shape
+    k_max = dest_pos.shape[1]
+    if dest_pos.shape[0] != T or tuple(topk_w.shape) != (T, k_max) or y.shape[1] != d or \
+            (shared is not None and tuple(shared.shape) != (T, d)):
+        raise ValueError("shape mismatch")
+    _check(load_library().moe_combine_bounded(_ptr(y), _ptr(topk_w), _ptr(dest_pos), _ptr(shared),
+                                              T, k_max, d, y.shape[0], _ptr(out), _ptr(d_status),
+                                              _stream(stream)), "moe_combine_bounded")

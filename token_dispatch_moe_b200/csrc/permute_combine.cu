@@ -22,15 +22,27 @@ namespace {
 
 constexpr int kRowWarps = 8;
 
-template <int U>
+// CHECK: every dest_pos outside [-1, rows) is skipped and reported (the
+// bounded entry points, and every launch of a MOE_CHECKED build).
+template <bool CHECK>
+__device__ __forceinline__ int checked_pos(int dp, int64_t rows, int32_t *status) {
+    if (CHECK && (dp < -1 || (int64_t)dp >= rows)) {
+        report(status, MOE_ERR_DEVICE_INDEX);
+        return -1;
+    }
+    return dp;
+}
+
+template <int U, bool CHECK>
 __global__ void __launch_bounds__(kRowWarps * 32)
     permute_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ dest_pos, int64_t T,
-                   int k_max, int nvec, uint4 *__restrict__ xs) {
+                   int k_max, int nvec, uint4 *__restrict__ xs, int64_t rows, int32_t *status) {
     const int lane = threadIdx.x & 31;
     const int64_t nw = (int64_t)gridDim.x * kRowWarps;
     griddep_wait();
     for (int64_t row = (int64_t)blockIdx.x * kRowWarps + (threadIdx.x >> 5); row < T; row += nw) {
-        const int dp = lane < k_max ? dest_pos[row * k_max + lane] : -1;
+        const int dp = checked_pos<CHECK>(lane < k_max ? dest_pos[row * k_max + lane] : -1, rows,
+                                          status);
         const uint4 *src = x + row * nvec;
         for (int v0 = 0; v0 < nvec; v0 += 32 * U) {
             uint4 buf[U];
@@ -54,17 +66,19 @@ __global__ void __launch_bounds__(kRowWarps * 32)
     griddep_launch_dependents();
 }
 
-template <int U>
+template <int U, bool CHECK>
 __global__ void __launch_bounds__(kRowWarps * 32)
     combine_kernel(const uint4 *__restrict__ y, const float *__restrict__ w,
                    const int32_t *__restrict__ dest_pos, const uint4 *__restrict__ shared,
-                   int64_t T, int k_max, int nvec, uint4 *__restrict__ out) {
+                   int64_t T, int k_max, int nvec, uint4 *__restrict__ out, int64_t rows,
+                   int32_t *status) {
     constexpr int J = 4;  // slots whose loads are issued together
     const int lane = threadIdx.x & 31;
     const int64_t nw = (int64_t)gridDim.x * kRowWarps;
     griddep_wait();
     for (int64_t row = (int64_t)blockIdx.x * kRowWarps + (threadIdx.x >> 5); row < T; row += nw) {
-        const int dp = lane < k_max ? dest_pos[row * k_max + lane] : -1;
+        const int dp = checked_pos<CHECK>(lane < k_max ? dest_pos[row * k_max + lane] : -1, rows,
+                                          status);
         const float wl = lane < k_max ? w[row * k_max + lane] : 0.0f;
         for (int v0 = 0; v0 < nvec; v0 += 32 * U) {
             float acc[U][8];
@@ -137,13 +151,13 @@ cudaError_t launch_rows(void (*kernel)(KArgs...), unsigned grid, cudaStream_t s,
     return cudaGetLastError();
 }
 
-}  // namespace
-}  // namespace moe
-
-extern "C" moe_status moe_permute(const moe_bf16_t *x, const int32_t *dest_pos, int64_t T,
-                                  int32_t k_max, int32_t d, moe_bf16_t *xs, moe_stream_t stream) {
-    using namespace moe;
-    if (T < 0 || k_max < 0 || k_max > 32 || d < 8 || d % 8 != 0) return MOE_ERR_INVALID_ARG;
+// Both row movers with the dest_pos check switched on (CHECK) or off.
+template <bool CHECK>
+moe_status run_permute(const moe_bf16_t *x, const int32_t *dest_pos, int64_t T, int32_t k_max,
+                       int32_t d, moe_bf16_t *xs, int64_t rows, int32_t *d_status,
+                       moe_stream_t stream) {
+    if (T < 0 || k_max < 0 || k_max > 32 || d < 8 || d % 8 != 0 || rows < 0)
+        return MOE_ERR_INVALID_ARG;
     if (T == 0 || k_max == 0) return MOE_OK;
     if (!x || !dest_pos || !xs || !aligned16(x) || !aligned16(xs)) return MOE_ERR_INVALID_ARG;
     if (T * (int64_t)k_max >= (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
@@ -152,10 +166,10 @@ extern "C" moe_status moe_permute(const moe_bf16_t *x, const int32_t *dest_pos, 
     const uint4 *x4 = reinterpret_cast<const uint4 *>(x);
     uint4 *xs4 = reinterpret_cast<uint4 *>(xs);
     const cudaError_t err =
-        d / 8 >= 512 ? launch_rows(permute_kernel<16>, row_grid(T), as_cuda(stream), x4, dest_pos,
-                                   T, (int)k_max, d / 8, xs4)
-                     : launch_rows(permute_kernel<8>, row_grid(T), as_cuda(stream), x4, dest_pos,
-                                   T, (int)k_max, d / 8, xs4);
+        d / 8 >= 512 ? launch_rows(permute_kernel<16, CHECK>, row_grid(T), as_cuda(stream), x4,
+                                   dest_pos, T, (int)k_max, d / 8, xs4, rows, d_status)
+                     : launch_rows(permute_kernel<8, CHECK>, row_grid(T), as_cuda(stream), x4,
+                                   dest_pos, T, (int)k_max, d / 8, xs4, rows, d_status);
     if (err != cudaSuccess) {
         cudaGetLastError();
         return MOE_ERR_CUDA;
@@ -163,11 +177,12 @@ extern "C" moe_status moe_permute(const moe_bf16_t *x, const int32_t *dest_pos, 
     return launch_status();
 }
 
-extern "C" moe_status moe_combine(const moe_bf16_t *y, const float *topk_w,
-                                  const int32_t *dest_pos, const moe_bf16_t *shared, int64_t T,
-                                  int32_t k_max, int32_t d, moe_bf16_t *out, moe_stream_t stream) {
-    using namespace moe;
-    if (T < 0 || k_max < 0 || k_max > 32 || d < 8 || d % 8 != 0) return MOE_ERR_INVALID_ARG;
+template <bool CHECK>
+moe_status run_combine(const moe_bf16_t *y, const float *topk_w, const int32_t *dest_pos,
+                       const moe_bf16_t *shared, int64_t T, int32_t k_max, int32_t d,
+                       moe_bf16_t *out, int64_t rows, int32_t *d_status, moe_stream_t stream) {
+    if (T < 0 || k_max < 0 || k_max > 32 || d < 8 || d % 8 != 0 || rows < 0)
+        return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if (!out || !aligned16(out) || (shared && !aligned16(shared))) return MOE_ERR_INVALID_ARG;
     if (k_max > 0 && (!y || !topk_w || !dest_pos || !aligned16(y))) return MOE_ERR_INVALID_ARG;
@@ -181,15 +196,56 @@ extern "C" moe_status moe_combine(const moe_bf16_t *y, const float *topk_w,
     const unsigned grid = row_grid(T);
     cudaStream_t cs = as_cuda(stream);
     const cudaError_t err =
-        nvec >= 128  ? launch_rows(combine_kernel<4>, grid, cs, y4, topk_w, dest_pos, s4, T,
-                                   (int)k_max, nvec, o4)
-        : nvec >= 64 ? launch_rows(combine_kernel<2>, grid, cs, y4, topk_w, dest_pos, s4, T,
-                                   (int)k_max, nvec, o4)
-                     : launch_rows(combine_kernel<1>, grid, cs, y4, topk_w, dest_pos, s4, T,
-                                   (int)k_max, nvec, o4);
+        nvec >= 128  ? launch_rows(combine_kernel<4, CHECK>, grid, cs, y4, topk_w, dest_pos, s4, T,
+                                   (int)k_max, nvec, o4, rows, d_status)
+        : nvec >= 64 ? launch_rows(combine_kernel<2, CHECK>, grid, cs, y4, topk_w, dest_pos, s4, T,
+                                   (int)k_max, nvec, o4, rows, d_status)
+                     : launch_rows(combine_kernel<1, CHECK>, grid, cs, y4, topk_w, dest_pos, s4, T,
+                                   (int)k_max, nvec, o4, rows, d_status);
     if (err != cudaSuccess) {
         cudaGetLastError();
         return MOE_ERR_CUDA;
     }
     return launch_status();
+}
+
+// A MOE_CHECKED build checks the plain entry points too, against T * k_max
+// rows (the most a dispatch of T tokens can fill); their signatures carry no
+// status word, so a skipped slot there is not reported.
+#ifdef MOE_CHECKED
+constexpr bool kCheckedBuild = true;
+#else
+constexpr bool kCheckedBuild = false;
+#endif
+
+}  // namespace
+}  // namespace moe
+
+extern "C" moe_status moe_permute(const moe_bf16_t *x, const int32_t *dest_pos, int64_t T,
+                                  int32_t k_max, int32_t d, moe_bf16_t *xs, moe_stream_t stream) {
+    return moe::run_permute<moe::kCheckedBuild>(x, dest_pos, T, k_max, d, xs, T * (int64_t)k_max,
+                                                nullptr, stream);
+}
+
+extern "C" moe_status moe_combine(const moe_bf16_t *y, const float *topk_w,
+                                  const int32_t *dest_pos, const moe_bf16_t *shared, int64_t T,
+                                  int32_t k_max, int32_t d, moe_bf16_t *out, moe_stream_t stream) {
+    return moe::run_combine<moe::kCheckedBuild>(y, topk_w, dest_pos, shared, T, k_max, d, out,
+                                                T * (int64_t)k_max, nullptr, stream);
+}
+
+extern "C" moe_status moe_permute_bounded(const moe_bf16_t *x, const int32_t *dest_pos, int64_t T,
+                                          int32_t k_max, int32_t d, moe_bf16_t *xs,
+                                          int64_t xs_rows, int32_t *d_status,
+                                          moe_stream_t stream) {
+    return moe::run_permute<true>(x, dest_pos, T, k_max, d, xs, xs_rows, d_status, stream);
+}
+
+extern "C" moe_status moe_combine_bounded(const moe_bf16_t *y, const float *topk_w,
+                                          const int32_t *dest_pos, const moe_bf16_t *shared,
+                                          int64_t T, int32_t k_max, int32_t d, int64_t y_rows,
+                                          moe_bf16_t *out, int32_t *d_status,
+                                          moe_stream_t stream) {
+    return moe::run_combine<true>(y, topk_w, dest_pos, shared, T, k_max, d, out, y_rows, d_status,
+                                  stream);
 }
