@@ -40,6 +40,10 @@ struct RouteArgs {
     int R;                    // rows per tile (multiple of 8)
     int64_t ntiles;
     int red_width;            // power of two >= k_max (width of the weight reductions)
+    // quad-per-row kernel (moe_route): padded row stride in floats, ring depth,
+    // values per lane of the warp-per-row routine (rows it takes over), row
+    // chunks of 16 experts, chunks per group
+    int rs, nstage, vpl, nch, cpg;
 };
 
 // Everything of RouteArgs that follows from the call's parameters (not the
@@ -83,6 +87,12 @@ inline void fill_route_args(RouteArgs &a, const float *logits, const float *bias
     a.red_width = width;
     a.R = 0;
     a.ntiles = 0;
+    a.vpl = vec ? 4 * ((E + 127) / 128) : (E + 31) / 32;
+    a.vpl = a.vpl <= 4 ? 4 : a.vpl <= 8 ? 8 : a.vpl <= 12 ? 12 : 16;
+    a.nch = (E + 15) / 16;
+    a.cpg = a.gsz % 16 == 0 ? a.gsz / 16 : 0;
+    a.rs = 0;
+    a.nstage = 0;
 }
 
 template <bool VEC>

@@ -30,7 +30,7 @@ def main(argv=None):
     ap.add_argument("--workload", required=True)
     ap.add_argument("--stage", required=True, choices=STAGES)
     ap.add_argument("--tokens", type=int, default=0)
-    ap.add_argument("--iters", type=int, default=20)
+    ap.add_argument("--iters", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--lib", default=None)
     args = ap.parse_args(argv)
@@ -82,23 +82,25 @@ def main(argv=None):
     torch.cuda.synchronize()
     if path.status.item() != 0:
         raise RuntimeError(f"device status {moe.moe_status_string(path.status.item())}")
+    from bench import ClockSampler, hash_stage_bytes, stage_bytes  # the bench's clocks, byte model
     times = []
-    for _ in range(args.iters):
-        flush.zero_()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        times.append(e0.elapsed_time(e1) * 1e3)
-    from bench import hash_stage_bytes, stage_bytes  # the bench's byte model
+    with ClockSampler(device.index) as clk:
+        for _ in range(args.iters):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            step()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1) * 1e3)
     model = hash_stage_bytes(wl) if st == "hash_route" else stage_bytes(wl, n_assign, fused)
     us = statistics.fmean(times)
     nbytes = model.get(st)
     print(json.dumps({
         "workload": wl.name, "tokens": wl.T, "stage": st, "lib": args.lib or "package",
         "us": round(us, 2), "us_min": round(min(times), 2), "iters": args.iters,
-        "bytes": nbytes, "GB_s": round(nbytes / (us * 1e-6) / 1e9, 1) if nbytes else None}))
+        "bytes": nbytes, "GB_s": round(nbytes / (us * 1e-6) / 1e9, 1) if nbytes else None,
+        "clocks": clk.summary()}))
 
 
 if __name__ == "__main__":
