@@ -234,7 +234,10 @@ def _dispatch(ids, E):
     (777, 16, 128, 0.4, False), (5000, 6, 384, 0.0, False), (20000, 32, 512, 0.1, True),
     (333, 3, 7, 0.2, False), (70000, 8, 256, 0.0, True),
     # 200 K slots: eight items a lane; E = 130: 33 quads of the segment-total rows
-    (25000, 8, 128, 0.3, True), (4000, 5, 130, 0.1, False)])
+    (25000, 8, 128, 0.3, True), (4000, 5, 130, 0.1, False),
+    # around the one-block launch (at most 1024 slots)
+    (128, 8, 64, 0.1, True), (1024, 1, 64, 0.1, True), (1025, 1, 16, 0.0, True),
+    (512, 8, 64, 0.1, True)])
 def test_dispatch_parity(T, k, E, empty_frac, hot):
     g = _gen(T + k + E)
     ids = torch.randint(0, E, (T, k), generator=g, device=DEV, dtype=torch.int32)

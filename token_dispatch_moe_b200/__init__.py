@@ -67,8 +67,10 @@ def library_path() -> str:
     return os.path.join(_PKG, _LIB_NAME)
 
 
-def load_library(path: str | None = None):
-    """Load (once) and return the ctypes handle of libmoe_dispatch.so."""
+def load_library(path: str | None = None, strict: bool = True):
+    """Load (once) and return the ctypes handle of libmoe_dispatch.so.  With a
+    path, load that build instead (not cached); strict=False there tolerates
+    an older build that lacks some entry points."""
     global _lib
     if _lib is not None and path is None:
         return _lib
@@ -103,6 +105,8 @@ def load_library(path: str | None = None):
         "moe_combine_bounded": ([P, P, P, P, i64, i32, i32, i64, P, P, P], st),
     }
     for name, (args, res) in sig.items():
+        if not strict and not hasattr(lib, name):
+            continue
         fn = getattr(lib, name)
         fn.argtypes = args
         fn.restype = res

@@ -40,7 +40,7 @@ def main(argv=None):
     from token_dispatch_moe_b200.workloads import WORKLOADS, make_inputs, num_assignments
 
     if args.lib:
-        moe._lib = moe.load_library(args.lib)
+        moe._lib = moe.load_library(args.lib, strict=False)
     moe.load_library()
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
