@@ -635,8 +635,7 @@ void *quad_fn_p(int P) {
         case 1: return (void *)route_quad_kernel<1, NCH>;
         case 2: return (void *)route_quad_kernel<2, NCH>;
         case 4: return (void *)route_quad_kernel<4, NCH>;
-        case 8: return (void *)route_quad_kernel<8, NCH>;
-        default: return (void *)route_quad_kernel<16, NCH>;
+        default: return (void *)route_quad_kernel<8, NCH>;
     }
 }
 
@@ -746,8 +745,11 @@ extern "C" moe_status moe_route(const float *logits, const float *bias, const in
     const bool vec = (E % 4 == 0);
     const int sms = sm_count();
 
-    // Quad-per-row kernel: 128-bit rows, k_max <= 16, groups of whole 16-expert chunks.
-    if (vec && p->k_max >= 1 && p->k_max <= 16 && (G == 1 || a.cpg > 0)) {
+    // Quad-per-row kernel: 128-bit rows, k_max <= 8, groups of whole 16-expert
+    // chunks.  A larger k_max keeps the warp-per-row kernel, whose top-k rounds
+    // follow each token's own k: with per-request k of 4, 8 or 16 over 128
+    // experts (qwen3_dynk) a network sized for 16 measured 30.7 against 20.5 us.
+    if (vec && p->k_max >= 1 && p->k_max <= 8 && (G == 1 || a.cpg > 0)) {
         const int nch_t = a.nch <= 8 ? 8 : a.nch <= 16 ? 16 : a.nch <= 24 ? 24 : 32;
         const size_t smem = (size_t)kQuadWarps * nch_t * 512 + (size_t)((E + 3) & ~3) * 4 +
                             (size_t)(kQuadThreads / 4) * kQuadGroupStride * 4 +
