@@ -392,10 +392,16 @@ def oracle_sample_size(wl, inp, budget_s: float, experts=None, hash_layer=False)
 
 
 # ----------------------------------------------------------------- our arm
+def dispatch_launches(n_slots: int) -> int:
+    """Kernels one dispatch launches: one block for at most 1024 slots, else
+    count + scatter."""
+    return 1 if n_slots <= 1024 else 2
+
+
 def chain_launches(wl, fused: bool) -> int:
     """Kernels of this library launched by one step of the chain."""
     gate_route = 1 if fused else (1 if wl.gate else 0) + 1
-    return gate_route + 2 + 1 + (1 if wl.combine else 0)
+    return gate_route + dispatch_launches(wl.T * wl.k_max) + 1 + (1 if wl.combine else 0)
 
 
 def run_ours(args):
@@ -647,7 +653,7 @@ def run_ours(args):
         "ms_per_step_stage_marked": round(statistics.fmean(m[-1] for m in marks), 5),
         "clocks": clk.summary(),
         "load": expert_load(path.counts), "env": host_env(device),
-        "gpu_launches": (5 if args.hash_layer else
+        "gpu_launches": (3 + dispatch_launches(wl.T * wl.k_max) if args.hash_layer else
                          chain_launches(wl, path.fused) + (2 if experts is not None else 0)) * K,
         "e2e": e2e,
     }
