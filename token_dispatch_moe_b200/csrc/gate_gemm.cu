@@ -533,6 +533,145 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ------------------------------------------------------- CTA-pair gate GEMM --
+// moe_gate_gemm for E <= 256 on pairs of CTAs (a cluster of two, on two SMs):
+// tcgen05.mma.cta_group::2 with M = 256, N = BN.  CTA r of a pair holds rows
+// 128r .. 128r + 127 of the pair's 256 rows of x and experts
+// r * BN/2 .. (r + 1) * BN/2 - 1 of W, at the same shared-memory offsets in
+// both CTAs, and its own 128 rows of the accumulator in its own TMEM.  So
+// each SM stages half of W per k-block instead of all of it.
+//   warp 0 (both CTAs)  TMA producer: waits for its own "empty" stage, then
+//                       loads its x rows and its half of W; both CTAs' loads
+//                       complete on the leader's "full" barrier, which the
+//                       leader arms with the bytes of both;
+//   warp 1 (leader)     MMA issuer; each commit arrives on the "empty"
+//                       barrier of that stage in both CTAs, the last one on
+//                       both CTAs' "accumulator ready" barrier;
+//   warp 2 (both)       TMEM allocation for the pair (cta_group::2);
+//   warps 4..7 (both)   epilogue: tcgen05.ld of its own 128 rows, fp32 stores.
+// A cluster barrier follows the barrier set-up (no commit or remote load can
+// reach a barrier before it is initialised) and precedes the TMEM free and
+// exit (no CTA leaves while the other may still read its shared memory or
+// signal its barriers).  Waits are bounded like gate_kernel's.
+__global__ void __launch_bounds__(kThreads, 1)
+    gate2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                 const GemmArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *const gbase = smem_raw + (base - raw);
+    const int S = a.stages;
+    const uint32_t bar0 = base + (uint32_t)S * a.stage_bytes;
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
+    const uint32_t tmem_full_bar = bar0 + 8u * (2 * S);
+    uint32_t *tmem_slot =
+        reinterpret_cast<uint32_t *>(gbase + (size_t)S * a.stage_bytes + 8u * (2 * S + 1));
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_cta_rank();
+    const bool leader = rank == 0;
+    const int m0 = (int)(blockIdx.x >> 1) * (2 * kBM) + (int)rank * kBM;
+    const int half = a.BN / 2;  // experts of W staged by each CTA
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        mbar_init(tmem_full_bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 2) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(a.tmem_cols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    griddep_wait();  // inputs and outputs are free of the previous kernel
+
+    if (warp == 0 && lane == 0) {
+        // TMA producer (both CTAs); the loads complete on the leader's barriers.
+        const uint32_t lead_full0 = cluster_map(full_bar(0), 0);
+        int issued = 0;
+        for (int kb = 0; kb < a.num_kb; ++kb) {
+            const int s = kb % S;
+            const uint32_t ph = (uint32_t)(kb / S) & 1u;
+            if (!mbar_wait(empty_bar(s), ph ^ 1u, a.status)) break;
+            const uint32_t st = base + (uint32_t)s * a.stage_bytes;
+            if (leader) mbar_arrive_expect_tx(full_bar(s), 2u * a.stage_bytes);
+            tma_load_2d_pair(st, &tmap_x, lead_full0 + 8u * s, kb * kBK, m0);
+            tma_load_2d_pair(st + kATileBytes, &tmap_w, lead_full0 + 8u * s, kb * kBK,
+                             (int)rank * half);
+            issued = kb + 1;
+        }
+        // Drain (leader: its full barriers count both CTAs' bytes).
+        if (leader)
+            for (int kb = issued - S < 0 ? 0 : issued - S; kb < issued; ++kb)
+                if (!mbar_wait(full_bar(kb % S), (uint32_t)(kb / S) & 1u, a.status)) break;
+    } else if (warp == 1 && lane == 0 && leader) {
+        // MMA issuer (leader only): M = 256 over the pair, N = BN.
+        for (int kb = 0; kb < a.num_kb; ++kb) {
+            const int s = kb % S;
+            const uint32_t ph = (uint32_t)(kb / S) & 1u;
+            if (!mbar_wait(full_bar(s), ph, a.status)) break;
+            tc_fence_after();
+            const uint32_t st = base + (uint32_t)s * a.stage_bytes;
+#pragma unroll
+            for (int k = 0; k < kBK / kUmmaK; ++k)
+                umma_bf16_pair(tmem_base, sw128_desc(st + (uint32_t)(k * kUmmaK * 2)),
+                               sw128_desc(st + kATileBytes + (uint32_t)(k * kUmmaK * 2)), a.idesc,
+                               (kb > 0 || k > 0) ? 1u : 0u);
+            umma_commit_pair(empty_bar(s));
+        }
+        // Both epilogues go once every MMA above has completed (also after a
+        // timeout, so that no epilogue reads a TMEM still being written).
+        umma_commit_pair(tmem_full_bar);
+    } else if (warp >= 4) {
+        const int q = warp & 3;
+        const bool ok = __all_sync(MOE_FULL_MASK, mbar_wait(tmem_full_bar, 0u, a.status));
+        tc_fence_after();
+        const int64_t row = (int64_t)m0 + q * 32 + lane;
+        const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16);
+        const bool vec = (a.E & 3) == 0;
+        if (ok) {
+            for (int c0 = 0; c0 < a.BN; c0 += 16) {
+                uint32_t r[16];
+                tmem_ld16(trow + (uint32_t)c0, r);
+                if (row < a.T) {
+                    float *dst = a.logits + row * a.E;
+                    if (vec && c0 + 16 <= a.E) {
+#pragma unroll
+                        for (int i = 0; i < 16; i += 4)
+                            *reinterpret_cast<float4 *>(dst + c0 + i) =
+                                make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
+                                            __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            if (c0 + i < a.E) dst[c0 + i] = __uint_as_float(r[i]);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    cluster_sync();
+    griddep_launch_dependents();
+    if (warp == 2) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(a.tmem_cols)
+                     : "memory");
+    }
+}
+
 // Shapes, stage count and shared-memory size of one launch.
 moe_status plan_gemm(int64_t T, int32_t d, int32_t E, size_t epi_bytes, GemmArgs &a,
                      size_t &smem) {
@@ -581,6 +720,70 @@ moe_status plan_gemm(int64_t T, int32_t d, int32_t E, size_t epi_bytes, GemmArgs
     a.stages = stages;
     smem = (size_t)stages * a.stage_bytes + overhead + epi_bytes;
     return MOE_OK;
+}
+
+// Shapes, stage count and shared-memory size of a CTA-pair launch (E <= 256).
+moe_status plan_pair(int64_t T, int32_t d, int32_t E, GemmArgs &a, size_t &smem) {
+    a.T = T;
+    a.E = E;
+    a.num_kb = (d + kBK - 1) / kBK;
+    a.NC = 1;
+    a.BN = (E + 15) / 16 * 16;  // each CTA stages BN/2 experts: a multiple of 8 rows
+    int cols = 32;
+    while (cols < a.BN) cols *= 2;
+    a.tmem_cols = cols;
+    a.stage_bytes = (uint32_t)(kATileBytes + (a.BN / 2) * 128);
+    // D fp32, A and B bf16, both K-major, N >> 3 at bit 17, M >> 4 at bit 24 (M = 256).
+    a.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(a.BN >> 3) << 17) |
+              ((uint32_t)((2 * kBM) >> 4) << 24);
+    int dev = 0, max_smem = 0, per_sm_smem = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&per_sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
+            cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    const int overhead = 1024 + 256;
+    const int static_smem = 1024;
+    int stages = (max_smem - static_smem - overhead) / (int)a.stage_bytes;
+    if (stages > 8) stages = 8;
+    // More CTAs than SMs: two CTAs an SM (each with half of its shared memory),
+    // so that one's epilogue and pipeline fill overlap the other's mainloop.
+    const int64_t ctas = 2 * ((T + 2 * kBM - 1) / (2 * kBM));
+    if (ctas > sm_count()) {
+        const int s2 = (per_sm_smem / 2 - 1024 - static_smem - overhead) / (int)a.stage_bytes;
+        if (s2 >= 2 && s2 < stages) stages = s2;
+    }
+    if (stages < 2) return MOE_ERR_UNSUPPORTED;
+    a.stages = stages;
+    smem = (size_t)stages * a.stage_bytes + overhead;
+    return MOE_OK;
+}
+
+moe_status launch_pair(const moe_bf16_t *x, const moe_bf16_t *w, const GemmArgs &a, size_t smem,
+                       int32_t d, moe_stream_t stream) {
+    CUtensorMap mx, mw;
+    if (!make_map(&mx, x, a.T, d, kBM) || !make_map(&mw, w, a.E, d, a.BN / 2)) return MOE_ERR_CUDA;
+    if (cudaFuncSetAttribute(gate2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    const unsigned grid = (unsigned)(2 * ((a.T + 2 * kBM - 1) / (2 * kBM)));
+    cudaLaunchAttribute attr[2];
+    cudaLaunchConfig_t cfg = pdl_config(dim3(grid), dim3(kThreads), smem, as_cuda(stream), attr);
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, gate2_kernel, mx, mw, a) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    return launch_status();
 }
 
 template <int MODE, int P, bool MONO = true, bool GROUPED = false>
@@ -640,6 +843,12 @@ extern "C" moe_status moe_gate_gemm(const moe_bf16_t *x, const moe_bf16_t *w, fl
     a.logits = logits;
     a.status = d_status;
     size_t smem = 0;
+    // Up to 256 experts (one accumulator): CTA pairs, each SM staging half of W.
+    if (E <= 256 && T > kBM) {
+        moe_status st = plan_pair(T, d, E, a, smem);
+        if (st != MOE_OK) return st;
+        return launch_pair(x, w, a, smem, d, stream);
+    }
     moe_status st = plan_gemm(T, d, E, 0, a, smem);
     if (st != MOE_OK) return st;
     FusedArgs f{};
