@@ -5,22 +5,32 @@
 // dtype.  bf16 x bf16 products are exact in fp32, so a bf16 tcgen05 MMA with an
 // fp32 accumulator computes the same quantity (up to summation order).
 //
-// sm_100a design (one 128-row M tile per CTA, the whole expert dimension as N):
-//   warp 0      TMA producer: 128x64 tile of x and Npad x64 tile of W per
-//               k-block into a ring of shared-memory stages, 128-byte swizzle,
-//               completion counted on a "full" mbarrier per stage;
-//   warp 1      MMA issuer (one thread): tcgen05.mma kind::f16, M=128, N=BN,
-//               K=16, A and B from shared memory through matrix descriptors,
-//               accumulator in TMEM; tcgen05.commit frees the stage ("empty"
-//               mbarrier) and, after the last k-block, signals the epilogue;
-//   warp 2      allocates / frees the TMEM accumulator columns;
+// sm_100a design: CTA pairs (clusters of two CTAs on two SMs, tcgen05
+// cta_group::2), one 256-row M tile per pair, the whole expert dimension as N.
+// CTA r of a pair stages rows 128r .. 128r + 127 of the tile's x and half of
+// the experts of each accumulator chunk, so each SM stages half of W per
+// k-block (deepseek_v3's gate: 250 -> 216 us against one 128-row tile per
+// CTA; qwen3_dynk's: 32.0 -> 27.5 us).
+//   warp 0      TMA producer (both CTAs): the x tile (128 x 64) and W halves
+//               (BN/2 x 64 per chunk) of each k-block into a ring of
+//               shared-memory stages, 128-byte swizzle; both CTAs' loads
+//               complete on the leader's "full" mbarrier of the stage;
+//   warp 1      MMA issuer (the leader's one thread): tcgen05.mma kind::f16,
+//               M=256, N=BN, K=16, A and B from both CTAs' shared memory
+//               through matrix descriptors (same offsets), each CTA's 128
+//               rows of the accumulator in its own TMEM; tcgen05.commit
+//               (multicast to both CTAs) frees the stage ("empty" mbarrier)
+//               and, after the last k-block, signals both epilogues;
+//   warp 2      allocates / frees the TMEM accumulator columns (both CTAs);
 //   warps 4..7  epilogue: tcgen05.ld (32 lanes x 16 columns per load), fp32
-//               stores of the logits rows.
+//               stores of the logits rows, or the route of each row
+//               (moe_gate_route).
 // E <= 256 is one accumulator of N = round16(E) columns; 256 < E <= 512 is two
 // of N = round16(E/2) side by side (UMMA N <= 256).  Rows beyond T and experts
 // beyond E are zero-filled by TMA and not stored.
 // Every mbarrier wait is bounded (about 2 s of %globaltimer); on expiry the
-// kernel records MOE_ERR_TIMEOUT, drains, frees its TMEM and returns.
+// kernel records MOE_ERR_TIMEOUT, drains, frees its TMEM and returns.  No TMA
+// load uses a cluster-wide multicast.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -396,7 +406,26 @@ __device__ __forceinline__ void route_epilogue(const GemmArgs &g, const FusedArg
 // MODE 0: the epilogue stores the logits.  MODE 1: it routes each row (and
 // stores the logits only if f.logits is set); MONO: keys are the logits;
 // GROUPED: a group limit applies.
-template <int MODE, int P, bool MONO = true, bool GROUPED = false>
+// The kernel runs as clusters of two CTAs on two SMs (tcgen05 cta_group::2,
+// M = 256 a pair).  CTA r of a pair holds rows 128r ..
+// 128r + 127 of the pair's 256 rows of x and, for each accumulator chunk c,
+// experts c*BN + r*BN/2 .. c*BN + (r+1)*BN/2 - 1 of W, at the same
+// shared-memory offsets in both CTAs, and its own 128 rows of the
+// accumulator in its own TMEM: each SM stages half of W per k-block.
+//   warp 0 (both CTAs)  waits for its own "empty" stage, then loads its x rows
+//                       and its halves of W; both CTAs' loads complete on the
+//                       leader's (rank 0) "full" barrier, which the leader
+//                       arms with the bytes of both;
+//   warp 1 (leader)     issues the MMAs; each commit arrives on that stage's
+//                       "empty" barrier in both CTAs, the last one on both
+//                       CTAs' "accumulator ready" barrier;
+//   warp 2 (both)       allocates the pair's TMEM (cta_group::2);
+//   warps 4..7 (both)   the epilogue on the CTA's own 128 rows.
+// A cluster barrier follows the barrier set-up (no commit or remote load
+// reaches a barrier before it is initialised) and precedes the TMEM free and
+// exit (no CTA leaves while the other may still read its shared memory or
+// signal its barriers).
+template <int MODE, int P, bool MONO, bool GROUPED, int NC>
 __global__ void __launch_bounds__(kThreads, 1)
     gate_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                 const GemmArgs a, const FusedArgs f) {
@@ -415,7 +444,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *epi = reinterpret_cast<float *>(gbase + (size_t)S * a.stage_bytes + 256);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * kBM;
+    const uint32_t rank = cluster_cta_rank();
+    const bool leader = rank == 0;
+    const int m0 = (int)(blockIdx.x >> 1) * (2 * kBM) + (int)rank * kBM;
+    const int half = a.BN / 2;  // experts of each accumulator chunk staged by each CTA
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -426,59 +458,62 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 2) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(tmem_slot)),
                      "r"(a.tmem_cols)
                      : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     griddep_wait();  // inputs and outputs are free of the previous kernel
 
     if (warp == 0 && lane == 0) {
-        // TMA producer.
+        // TMA producer; the loads complete on the leader's barriers.
+        const uint32_t lead_full0 = cluster_map(full_bar(0), 0);
         int issued = 0;
         for (int kb = 0; kb < a.num_kb; ++kb) {
             const int s = kb % S;
             const uint32_t ph = (uint32_t)(kb / S) & 1u;
             if (!mbar_wait(empty_bar(s), ph ^ 1u, a.status)) break;
             const uint32_t st = base + (uint32_t)s * a.stage_bytes;
-            mbar_arrive_expect_tx(full_bar(s), a.stage_bytes);
-            tma_load_2d(st, &tmap_x, full_bar(s), kb * kBK, m0);
-            for (int c = 0; c < a.NC; ++c)
-                tma_load_2d(st + kATileBytes + (uint32_t)(c * a.BN * 128), &tmap_w, full_bar(s),
-                            kb * kBK, c * a.BN);
+            if (leader) mbar_arrive_expect_tx(full_bar(s), 2u * a.stage_bytes);
+            tma_load_2d_pair(st, &tmap_x, lead_full0 + 8u * s, kb * kBK, m0);
+            for (int c = 0; c < NC; ++c)
+                tma_load_2d_pair(st + kATileBytes + (uint32_t)(c * half * 128), &tmap_w,
+                                 lead_full0 + 8u * s, kb * kBK, c * a.BN + (int)rank * half);
             issued = kb + 1;
         }
-        // Drain: every stage's last issued load has landed before the CTA exits.
-        for (int kb = issued - S < 0 ? 0 : issued - S; kb < issued; ++kb)
-            if (!mbar_wait(full_bar(kb % S), (uint32_t)(kb / S) & 1u, a.status)) break;
+        // Drain (leader: its full barriers count both CTAs' bytes).
+        if (leader)
+            for (int kb = issued - S < 0 ? 0 : issued - S; kb < issued; ++kb)
+                if (!mbar_wait(full_bar(kb % S), (uint32_t)(kb / S) & 1u, a.status)) break;
     } else if (warp == 1 && lane == 0) {
-        // MMA issuer.
-        for (int kb = 0; kb < a.num_kb; ++kb) {
-            const int s = kb % S;
-            const uint32_t ph = (uint32_t)(kb / S) & 1u;
-            if (!mbar_wait(full_bar(s), ph, a.status)) break;
-            tc_fence_after();
-            const uint32_t st = base + (uint32_t)s * a.stage_bytes;
+        // MMA issuer: the leader alone, M = 256, N = BN per chunk.
+        if (leader) {
+            for (int kb = 0; kb < a.num_kb; ++kb) {
+                const int s = kb % S;
+                const uint32_t ph = (uint32_t)(kb / S) & 1u;
+                if (!mbar_wait(full_bar(s), ph, a.status)) break;
+                tc_fence_after();
+                const uint32_t st = base + (uint32_t)s * a.stage_bytes;
 #pragma unroll
-            for (int k = 0; k < kBK / kUmmaK; ++k) {
-                const uint64_t adesc = sw128_desc(st + (uint32_t)(k * kUmmaK * 2));
-                for (int c = 0; c < a.NC; ++c) {
-                    const uint64_t bdesc = sw128_desc(st + kATileBytes +
-                                                      (uint32_t)(c * a.BN * 128 + k * kUmmaK * 2));
-                    umma_bf16(tmem_base + (uint32_t)(c * a.BN), adesc, bdesc, a.idesc,
-                              (kb > 0 || k > 0) ? 1u : 0u);
+                for (int k = 0; k < kBK / kUmmaK; ++k) {
+                    const uint64_t adesc = sw128_desc(st + (uint32_t)(k * kUmmaK * 2));
+                    for (int c = 0; c < NC; ++c)
+                        umma_bf16_pair(tmem_base + (uint32_t)(c * a.BN), adesc,
+                                       sw128_desc(st + kATileBytes +
+                                                  (uint32_t)(c * half * 128 + k * kUmmaK * 2)),
+                                       a.idesc, (kb > 0 || k > 0) ? 1u : 0u);
                 }
+                umma_commit_pair(empty_bar(s));
             }
-            umma_commit(empty_bar(s));
+            // Both epilogues go once every MMA above has completed (also after
+            // a timeout, so that no epilogue reads a TMEM still being written).
+            umma_commit_pair(tmem_full_bar);
         }
-        // Signals the epilogue once every MMA issued above has completed (also
-        // on the timeout path, so the epilogue never reads a TMEM in use).
-        umma_commit(tmem_full_bar);
     } else if (warp >= 4) {
         // Epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = tile rows.
         const int q = warp & 3;
@@ -490,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (MODE == 0) {
             const bool vec = (a.E & 3) == 0;
             if (ok) {
-                const int ncols = a.NC * a.BN;
+                const int ncols = NC * a.BN;
                 for (int c0 = 0; c0 < ncols; c0 += 16) {
                     uint32_t r[16];
                     tmem_ld16(trow + (uint32_t)c0, r);
@@ -523,145 +558,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     tc_fence_before();
-    __syncthreads();
-    griddep_launch_dependents();
-    if (warp == 2) {
-        tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                     "r"(a.tmem_cols)
-                     : "memory");
-    }
-}
-
-// ------------------------------------------------------- CTA-pair gate GEMM --
-// moe_gate_gemm for E <= 256 on pairs of CTAs (a cluster of two, on two SMs):
-// tcgen05.mma.cta_group::2 with M = 256, N = BN.  CTA r of a pair holds rows
-// 128r .. 128r + 127 of the pair's 256 rows of x and experts
-// r * BN/2 .. (r + 1) * BN/2 - 1 of W, at the same shared-memory offsets in
-// both CTAs, and its own 128 rows of the accumulator in its own TMEM.  So
-// each SM stages half of W per k-block instead of all of it.
-//   warp 0 (both CTAs)  TMA producer: waits for its own "empty" stage, then
-//                       loads its x rows and its half of W; both CTAs' loads
-//                       complete on the leader's "full" barrier, which the
-//                       leader arms with the bytes of both;
-//   warp 1 (leader)     MMA issuer; each commit arrives on the "empty"
-//                       barrier of that stage in both CTAs, the last one on
-//                       both CTAs' "accumulator ready" barrier;
-//   warp 2 (both)       TMEM allocation for the pair (cta_group::2);
-//   warps 4..7 (both)   epilogue: tcgen05.ld of its own 128 rows, fp32 stores.
-// A cluster barrier follows the barrier set-up (no commit or remote load can
-// reach a barrier before it is initialised) and precedes the TMEM free and
-// exit (no CTA leaves while the other may still read its shared memory or
-// signal its barriers).  Waits are bounded like gate_kernel's.
-__global__ void __launch_bounds__(kThreads, 1)
-    gate2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                 const GemmArgs a) {
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t base = (raw + 1023u) & ~1023u;
-    uint8_t *const gbase = smem_raw + (base - raw);
-    const int S = a.stages;
-    const uint32_t bar0 = base + (uint32_t)S * a.stage_bytes;
-    auto full_bar = [&](int s) { return bar0 + 8u * s; };
-    auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
-    const uint32_t tmem_full_bar = bar0 + 8u * (2 * S);
-    uint32_t *tmem_slot =
-        reinterpret_cast<uint32_t *>(gbase + (size_t)S * a.stage_bytes + 8u * (2 * S + 1));
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_cta_rank();
-    const bool leader = rank == 0;
-    const int m0 = (int)(blockIdx.x >> 1) * (2 * kBM) + (int)rank * kBM;
-    const int half = a.BN / 2;  // experts of W staged by each CTA
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), 1);
-        }
-        mbar_init(tmem_full_bar, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    if (warp == 2) {
-        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                         smem_u32(tmem_slot)),
-                     "r"(a.tmem_cols)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-    }
-    tc_fence_before();
-    cluster_sync();
-    tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
-    griddep_wait();  // inputs and outputs are free of the previous kernel
-
-    if (warp == 0 && lane == 0) {
-        // TMA producer (both CTAs); the loads complete on the leader's barriers.
-        const uint32_t lead_full0 = cluster_map(full_bar(0), 0);
-        int issued = 0;
-        for (int kb = 0; kb < a.num_kb; ++kb) {
-            const int s = kb % S;
-            const uint32_t ph = (uint32_t)(kb / S) & 1u;
-            if (!mbar_wait(empty_bar(s), ph ^ 1u, a.status)) break;
-            const uint32_t st = base + (uint32_t)s * a.stage_bytes;
-            if (leader) mbar_arrive_expect_tx(full_bar(s), 2u * a.stage_bytes);
-            tma_load_2d_pair(st, &tmap_x, lead_full0 + 8u * s, kb * kBK, m0);
-            tma_load_2d_pair(st + kATileBytes, &tmap_w, lead_full0 + 8u * s, kb * kBK,
-                             (int)rank * half);
-            issued = kb + 1;
-        }
-        // Drain (leader: its full barriers count both CTAs' bytes).
-        if (leader)
-            for (int kb = issued - S < 0 ? 0 : issued - S; kb < issued; ++kb)
-                if (!mbar_wait(full_bar(kb % S), (uint32_t)(kb / S) & 1u, a.status)) break;
-    } else if (warp == 1 && lane == 0 && leader) {
-        // MMA issuer (leader only): M = 256 over the pair, N = BN.
-        for (int kb = 0; kb < a.num_kb; ++kb) {
-            const int s = kb % S;
-            const uint32_t ph = (uint32_t)(kb / S) & 1u;
-            if (!mbar_wait(full_bar(s), ph, a.status)) break;
-            tc_fence_after();
-            const uint32_t st = base + (uint32_t)s * a.stage_bytes;
-#pragma unroll
-            for (int k = 0; k < kBK / kUmmaK; ++k)
-                umma_bf16_pair(tmem_base, sw128_desc(st + (uint32_t)(k * kUmmaK * 2)),
-                               sw128_desc(st + kATileBytes + (uint32_t)(k * kUmmaK * 2)), a.idesc,
-                               (kb > 0 || k > 0) ? 1u : 0u);
-            umma_commit_pair(empty_bar(s));
-        }
-        // Both epilogues go once every MMA above has completed (also after a
-        // timeout, so that no epilogue reads a TMEM still being written).
-        umma_commit_pair(tmem_full_bar);
-    } else if (warp >= 4) {
-        const int q = warp & 3;
-        const bool ok = __all_sync(MOE_FULL_MASK, mbar_wait(tmem_full_bar, 0u, a.status));
-        tc_fence_after();
-        const int64_t row = (int64_t)m0 + q * 32 + lane;
-        const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16);
-        const bool vec = (a.E & 3) == 0;
-        if (ok) {
-            for (int c0 = 0; c0 < a.BN; c0 += 16) {
-                uint32_t r[16];
-                tmem_ld16(trow + (uint32_t)c0, r);
-                if (row < a.T) {
-                    float *dst = a.logits + row * a.E;
-                    if (vec && c0 + 16 <= a.E) {
-#pragma unroll
-                        for (int i = 0; i < 16; i += 4)
-                            *reinterpret_cast<float4 *>(dst + c0 + i) =
-                                make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
-                                            __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            if (c0 + i < a.E) dst[c0 + i] = __uint_as_float(r[i]);
-                    }
-                }
-            }
-        }
-    }
-
-    tc_fence_before();
     cluster_sync();
     griddep_launch_dependents();
     if (warp == 2) {
@@ -686,10 +582,12 @@ moe_status plan_gemm(int64_t T, int32_t d, int32_t E, size_t epi_bytes, GemmArgs
     int cols = 32;
     while (cols < npad) cols *= 2;
     a.tmem_cols = cols;
-    a.stage_bytes = (uint32_t)(kATileBytes + npad * 128);
-    // D fp32, A and B bf16, both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+    // Each CTA of a pair stages its 128 rows of x and half of each chunk's experts.
+    a.stage_bytes = (uint32_t)(kATileBytes + a.NC * (a.BN / 2) * 128);
+    // D fp32, A and B bf16, both K-major, N >> 3 at bit 17, M >> 4 at bit 24
+    // (M = 256: the pair's two 128-row halves).
     a.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(a.BN >> 3) << 17) |
-              ((uint32_t)(kBM >> 4) << 24);
+              ((uint32_t)((2 * kBM) >> 4) << 24);
     int dev = 0, max_smem = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
@@ -703,11 +601,11 @@ moe_status plan_gemm(int64_t T, int32_t d, int32_t E, size_t epi_bytes, GemmArgs
                        (int)a.stage_bytes);
     if (stages > 8) stages = 8;
     if (stages < 2) return MOE_ERR_UNSUPPORTED;
-    // More tiles than SMs (several waves), a plain epilogue and at most half of
+    // More CTAs than SMs (several waves), a plain epilogue and at most half of
     // the TMEM: two CTAs per SM, so that one's epilogue and pipeline fill
-    // overlap the other's mainloop (deepseek_v3's gate: 328 -> 253 us), with
-    // as many stages as half of the SM's shared memory holds.
-    const int64_t tiles = (T + kBM - 1) / kBM;
+    // overlap the other's mainloop, with as many stages as half of the SM's
+    // shared memory holds.
+    const int64_t tiles = 2 * ((T + 2 * kBM - 1) / (2 * kBM));
     int per_sm_smem = 0;
     if (epi_bytes == 0 && a.tmem_cols <= 256 && tiles > sm_count() &&
         cudaDeviceGetAttribute(&per_sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) ==
@@ -722,55 +620,19 @@ moe_status plan_gemm(int64_t T, int32_t d, int32_t E, size_t epi_bytes, GemmArgs
     return MOE_OK;
 }
 
-// Shapes, stage count and shared-memory size of a CTA-pair launch (E <= 256).
-moe_status plan_pair(int64_t T, int32_t d, int32_t E, GemmArgs &a, size_t &smem) {
-    a.T = T;
-    a.E = E;
-    a.num_kb = (d + kBK - 1) / kBK;
-    a.NC = 1;
-    a.BN = (E + 15) / 16 * 16;  // each CTA stages BN/2 experts: a multiple of 8 rows
-    int cols = 32;
-    while (cols < a.BN) cols *= 2;
-    a.tmem_cols = cols;
-    a.stage_bytes = (uint32_t)(kATileBytes + (a.BN / 2) * 128);
-    // D fp32, A and B bf16, both K-major, N >> 3 at bit 17, M >> 4 at bit 24 (M = 256).
-    a.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(a.BN >> 3) << 17) |
-              ((uint32_t)((2 * kBM) >> 4) << 24);
-    int dev = 0, max_smem = 0, per_sm_smem = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
-            cudaSuccess ||
-        cudaDeviceGetAttribute(&per_sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
-            cudaSuccess) {
-        cudaGetLastError();
-        return MOE_ERR_CUDA;
-    }
-    const int overhead = 1024 + 256;
-    const int static_smem = 1024;
-    int stages = (max_smem - static_smem - overhead) / (int)a.stage_bytes;
-    if (stages > 8) stages = 8;
-    // More CTAs than SMs: two CTAs an SM (each with half of its shared memory),
-    // so that one's epilogue and pipeline fill overlap the other's mainloop.
-    const int64_t ctas = 2 * ((T + 2 * kBM - 1) / (2 * kBM));
-    if (ctas > sm_count()) {
-        const int s2 = (per_sm_smem / 2 - 1024 - static_smem - overhead) / (int)a.stage_bytes;
-        if (s2 >= 2 && s2 < stages) stages = s2;
-    }
-    if (stages < 2) return MOE_ERR_UNSUPPORTED;
-    a.stages = stages;
-    smem = (size_t)stages * a.stage_bytes + overhead;
-    return MOE_OK;
-}
-
-moe_status launch_pair(const moe_bf16_t *x, const moe_bf16_t *w, const GemmArgs &a, size_t smem,
-                       int32_t d, moe_stream_t stream) {
+// The chunk count is a template argument: a runtime loop over it in the MMA
+// issue measured 5 us slower at qwen3_dynk (30.6 against 26.5 us).
+template <int MODE, int P, bool MONO, bool GROUPED, int NC>
+moe_status launch_gate_nc(const moe_bf16_t *x, const moe_bf16_t *w, const GemmArgs &a,
+                       const FusedArgs &f, size_t smem, int32_t d, moe_stream_t stream) {
     CUtensorMap mx, mw;
     if (!make_map(&mx, x, a.T, d, kBM) || !make_map(&mw, w, a.E, d, a.BN / 2)) return MOE_ERR_CUDA;
-    if (cudaFuncSetAttribute(gate2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess) {
+    if (cudaFuncSetAttribute(gate_kernel<MODE, P, MONO, GROUPED, NC>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
         cudaGetLastError();
         return MOE_ERR_CUDA;
     }
+    // One pair of CTAs (a cluster of two) per 256 rows.
     const unsigned grid = (unsigned)(2 * ((a.T + 2 * kBM - 1) / (2 * kBM)));
     cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = pdl_config(dim3(grid), dim3(kThreads), smem, as_cuda(stream), attr);
@@ -779,7 +641,7 @@ moe_status launch_pair(const moe_bf16_t *x, const moe_bf16_t *w, const GemmArgs 
     attr[1].val.clusterDim.y = 1;
     attr[1].val.clusterDim.z = 1;
     cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, gate2_kernel, mx, mw, a) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, gate_kernel<MODE, P, MONO, GROUPED, NC>, mx, mw, a, f) != cudaSuccess) {
         cudaGetLastError();
         return MOE_ERR_CUDA;
     }
@@ -789,20 +651,8 @@ moe_status launch_pair(const moe_bf16_t *x, const moe_bf16_t *w, const GemmArgs 
 template <int MODE, int P, bool MONO = true, bool GROUPED = false>
 moe_status launch_gate(const moe_bf16_t *x, const moe_bf16_t *w, const GemmArgs &a,
                        const FusedArgs &f, size_t smem, int32_t d, moe_stream_t stream) {
-    CUtensorMap mx, mw;
-    if (!make_map(&mx, x, a.T, d, kBM) || !make_map(&mw, w, a.E, d, a.BN)) return MOE_ERR_CUDA;
-    if (cudaFuncSetAttribute(gate_kernel<MODE, P, MONO, GROUPED>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
-        cudaGetLastError();
-        return MOE_ERR_CUDA;
-    }
-    const unsigned grid = (unsigned)((a.T + kBM - 1) / kBM);
-    if (launch_pdl(gate_kernel<MODE, P, MONO, GROUPED>, dim3(grid), dim3(kThreads), smem,
-                   as_cuda(stream), mx, mw, a, f) != cudaSuccess) {
-        cudaGetLastError();
-        return MOE_ERR_CUDA;
-    }
-    return launch_status();
+    return a.NC == 1 ? launch_gate_nc<MODE, P, MONO, GROUPED, 1>(x, w, a, f, smem, d, stream)
+                     : launch_gate_nc<MODE, P, MONO, GROUPED, 2>(x, w, a, f, smem, d, stream);
 }
 
 template <bool MONO, bool GROUPED>
@@ -843,12 +693,6 @@ extern "C" moe_status moe_gate_gemm(const moe_bf16_t *x, const moe_bf16_t *w, fl
     a.logits = logits;
     a.status = d_status;
     size_t smem = 0;
-    // Up to 256 experts (one accumulator): CTA pairs, each SM staging half of W.
-    if (E <= 256 && T > kBM) {
-        moe_status st = plan_pair(T, d, E, a, smem);
-        if (st != MOE_OK) return st;
-        return launch_pair(x, w, a, smem, d, stream);
-    }
     moe_status st = plan_gemm(T, d, E, 0, a, smem);
     if (st != MOE_OK) return st;
     FusedArgs f{};
