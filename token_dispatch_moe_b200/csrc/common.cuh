@@ -89,6 +89,18 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
+// Selection key of the sigmoid score, shared by every routing kernel so that
+// they agree bit for bit: 1 / (1 + e^-l) with accurate expf and the hardware
+// reciprocal (rcp.approx: at most 1 ulp from the correctly rounded value, a
+// relative 6e-8, far inside the 1e-6 band within which the parity rule lets
+// near-tied experts swap; its argument is >= 1 and its result in (0, 1], so
+// flushing subnormals changes nothing).  Weights use sigmoid_score below.
+__device__ __forceinline__ float sigmoid_key(float l) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + expf(-l)));
+    return r;
+}
+
 // Per-expert scores that do not depend on the rest of the row.
 __device__ __forceinline__ float sigmoid_score(float l) { return 1.0f / (1.0f + expf(-l)); }
 __device__ __forceinline__ float sqrt_softplus_score(float l) {

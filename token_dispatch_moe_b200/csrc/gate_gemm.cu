@@ -93,7 +93,7 @@ __device__ __forceinline__ float fused_key(const FusedArgs &f, float l, int e, c
     if (f.score == MOE_SCORE_SOFTMAX)
         x = expf(l - st.m) * zinv;
     else if (f.score == MOE_SCORE_SIGMOID)
-        x = __frcp_rn(1.0f + expf(-l));
+        x = sigmoid_key(l);
     else if (f.score == MOE_SCORE_SQRT_SOFTPLUS)
         x = sqrt_softplus_score(l);
     else

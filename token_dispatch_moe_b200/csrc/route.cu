@@ -322,7 +322,7 @@ __device__ __forceinline__ float quad_key(int score, float l, float m, float zin
     if (score == MOE_SCORE_SOFTMAX)
         x = expf(l - m) * zinv;
     else if (score == MOE_SCORE_SIGMOID)
-        x = __frcp_rn(1.0f + expf(-l));
+        x = sigmoid_key(l);
     else if (score == MOE_SCORE_SQRT_SOFTPLUS)
         x = sqrt_softplus_score(l);
     return x + b;

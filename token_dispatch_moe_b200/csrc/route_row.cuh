@@ -248,7 +248,7 @@ __device__ __forceinline__ void route_row(const RouteArgs &a, const float *src, 
             if (a.score == MOE_SCORE_SOFTMAX)
                 x = expf(l[s] - m) * zinv;
             else if (a.score == MOE_SCORE_SIGMOID)
-                x = __frcp_rn(1.0f + expf(-l[s]));
+                x = sigmoid_key(l[s]);
             else if (a.score == MOE_SCORE_SQRT_SOFTPLUS)
                 x = sqrt_softplus_score(l[s]);
             v[s] = x + biasr[s];
@@ -437,7 +437,7 @@ __device__ __forceinline__ void route_row_top1(const RouteArgs &a, const float *
             if (a.score == MOE_SCORE_SOFTMAX)
                 v = expf(l[s] - m) * zinv;
             else if (a.score == MOE_SCORE_SIGMOID)
-                v = __frcp_rn(1.0f + expf(-l[s]));
+                v = sigmoid_key(l[s]);
             else if (a.score == MOE_SCORE_SQRT_SOFTPLUS)
                 v = sqrt_softplus_score(l[s]);
             v += biasr[s];
