@@ -192,6 +192,38 @@ def test_hash_route_parity(score, with_logits, renorm):
     assert np.all(np.abs(wg - o["w"]) <= 1e-5 * np.abs(o["w"]))
 
 
+@pytest.mark.parametrize("T,k,score,renorm", [(1001, 1, "softmax", True),
+                                               (1001, 4, "sigmoid", False),
+                                               (1001, 5, "sqrt_softplus", True),
+                                               (1001, 8, "topk_softmax", True),
+                                               (1001, 9, "softmax", True),
+                                               (1001, 16, "sigmoid", True),
+                                               (1001, 17, "sqrt_softplus", False),
+                                               (1001, 32, "softmax", True),
+                                               (200003, 2, "sqrt_softplus", True)])
+def test_hash_route_lanes_per_token(T, k, score, renorm):
+    """Every lane width (4, 8, 16, 32 lanes a token), a ragged last warp and,
+    at 200003 tokens, more rows than one pass of the grid."""
+    E, vocab = 64, 3000
+    g = _gen(100 + k)
+    tok = torch.randint(0, vocab, (T,), generator=g, device=DEV, dtype=torch.int32)
+    table = torch.randint(0, E, (vocab, k), generator=g, device=DEV, dtype=torch.int32)
+    logits = torch.randn((T, E), generator=g, device=DEV)
+    p = moe.RouteParams.make(E, k, score, renormalize=renorm, route_scale=0.75)
+    ids = torch.full((T, k), -9, dtype=torch.int32, device=DEV)
+    w = torch.full((T, k), -9.0, device=DEV)
+    st = _status()
+    moe.moe_hash_route(tok, table, logits, p, ids, w, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    o = oracle.hash_route(tok.cpu().numpy(), table.cpu().numpy(), num_experts=E,
+                          logits=logits.cpu().numpy(), score=oracle_score(score),
+                          renormalize=renorm, route_scale=0.75)
+    assert np.array_equal(ids.cpu().numpy(), o["ids"])
+    wg = w.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(wg - o["w"]) <= 1e-5 * np.abs(o["w"]))
+
+
 def oracle_score(name):
     return {"softmax": oracle.SOFTMAX, "sigmoid": oracle.SIGMOID,
             "sqrt_softplus": oracle.SQRT_SOFTPLUS, "topk_softmax": oracle.TOPK_SOFTMAX}[name]

@@ -713,6 +713,67 @@ __global__ void __launch_bounds__(256) hash_route_kernel(const HashArgs a) {
     }
 }
 
+// W lanes per token, 32 / W tokens a warp (W = the power of two >= k, at most
+// 32): every token's dependent loads (token id, table row, logits of the
+// looked-up experts) are in flight together with those of the warp's other
+// tokens.  Scores that need only the looked-up logits; a softmax over the
+// whole row without renormalisation takes hash_route_kernel.
+template <int W>
+__global__ void __launch_bounds__(256) hash_route_grouped_kernel(const HashArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int sl = lane & (W - 1);  // slot of this lane in its token
+    constexpr int TPW = 32 / W;     // tokens per warp
+    const int64_t step = (int64_t)gridDim.x * (blockDim.x >> 5) * TPW;
+    griddep_wait();
+    for (int64_t row0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * TPW;
+         row0 < a.T; row0 += step) {
+        const int64_t row = row0 + lane / W;
+        const bool live = row < a.T;
+        const int v = live ? a.tok[row] : 0;
+        const bool row_ok = live && v >= 0 && v < a.vocab;
+        if (live && !row_ok && sl == 0) report(a.status, MOE_ERR_DEVICE_INDEX);
+        int id = -1;
+        if (row_ok && sl < a.k) {
+            id = a.table[(int64_t)v * a.k + sl];
+            if (id < 0 || id >= a.E) {
+                report(a.status, MOE_ERR_DEVICE_INDEX);
+                id = -1;
+            }
+        }
+        const bool act = id >= 0;
+        float s;
+        if (a.logits) {
+            const float l = act ? a.logits[row * a.E + id] : 0.0f;
+            if (l != l) report(a.status, MOE_ERR_NAN_LOGIT);
+            if (a.score == MOE_SCORE_SOFTMAX || a.score == MOE_SCORE_TOPK_SOFTMAX) {
+                float msel = act ? l : -INFINITY;
+#pragma unroll
+                for (int o = 1; o < W; o <<= 1)
+                    msel = fmaxf(msel, __shfl_xor_sync(MOE_FULL_MASK, msel, o));
+                s = act ? expf(l - msel) : 0.0f;
+            } else if (a.score == MOE_SCORE_SIGMOID) {
+                s = act ? sigmoid_score(l) : 0.0f;
+            } else {
+                s = act ? sqrt_softplus_score(l) : 0.0f;
+            }
+            if (a.renorm || a.score == MOE_SCORE_TOPK_SOFTMAX) {
+                float sum = s;
+#pragma unroll
+                for (int o = 1; o < W; o <<= 1) sum += __shfl_xor_sync(MOE_FULL_MASK, sum, o);
+                if (act && sum > 0.0f) s = s / sum;
+            }
+            s *= a.scale;
+        } else {
+            s = act ? a.scale / (float)a.k : 0.0f;
+        }
+        if (live && sl < a.k) {
+            a.ids[row * a.k + sl] = id;
+            a.w[row * a.k + sl] = act ? s : 0.0f;
+        }
+    }
+    griddep_launch_dependents();
+}
+
 bool valid_score(int s) {
     return s == MOE_SCORE_SOFTMAX || s == MOE_SCORE_SIGMOID || s == MOE_SCORE_SQRT_SOFTPLUS ||
            s == MOE_SCORE_TOPK_SOFTMAX;
@@ -851,9 +912,28 @@ extern "C" moe_status moe_hash_route(const int32_t *token_ids, const int32_t *ti
     a.score = p->score;
     a.renorm = p->renormalize ? 1 : 0;
     a.scale = p->route_scale;
-    const int64_t blocks_needed = (T + 7) / 8;
     const int64_t cap = (int64_t)sm_count() * 8;
-    hash_route_kernel<<<(unsigned)(blocks_needed < cap ? blocks_needed : cap), 256, 0,
-                        as_cuda(stream)>>>(a);
+    if (logits && p->score == MOE_SCORE_SOFTMAX && !p->renormalize) {
+        // full-row softmax statistics: one warp a token
+        const int64_t blocks_needed = (T + 7) / 8;
+        hash_route_kernel<<<(unsigned)(blocks_needed < cap ? blocks_needed : cap), 256, 0,
+                            as_cuda(stream)>>>(a);
+        return launch_status();
+    }
+    const int W = k <= 4 ? 4 : k <= 8 ? 8 : k <= 16 ? 16 : 32;
+    const int64_t per_block = 8 * (32 / W);
+    const int64_t blocks_needed = (T + per_block - 1) / per_block;
+    const unsigned grid = (unsigned)(blocks_needed < cap ? blocks_needed : cap);
+    cudaError_t err;
+    switch (W) {
+        case 4: err = launch_pdl(hash_route_grouped_kernel<4>, dim3(grid), dim3(256), 0, as_cuda(stream), a); break;
+        case 8: err = launch_pdl(hash_route_grouped_kernel<8>, dim3(grid), dim3(256), 0, as_cuda(stream), a); break;
+        case 16: err = launch_pdl(hash_route_grouped_kernel<16>, dim3(grid), dim3(256), 0, as_cuda(stream), a); break;
+        default: err = launch_pdl(hash_route_grouped_kernel<32>, dim3(grid), dim3(256), 0, as_cuda(stream), a); break;
+    }
+    if (err != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
     return launch_status();
 }
