@@ -107,6 +107,24 @@ __device__ __forceinline__ float sqrt_softplus_score(float l) {
     return sqrtf(fmaxf(l, 0.0f) + log1pf(expf(-fabsf(l))));
 }
 
+// Selection keys of N logits in place, before the bias: the score function is
+// chosen once for the whole array (a branch per logit costs more than the key
+// itself).  m and zinv are the row's max and 1 / softmax denominator (read for
+// softmax only); the gpt-oss score and monotone keys leave the logits as they are.
+template <int N>
+__device__ __forceinline__ void score_keys(int score, float (&x)[N], float m, float zinv) {
+    if (score == MOE_SCORE_SIGMOID) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) x[i] = sigmoid_key(x[i]);
+    } else if (score == MOE_SCORE_SQRT_SOFTPLUS) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) x[i] = sqrt_softplus_score(x[i]);
+    } else if (score == MOE_SCORE_SOFTMAX) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) x[i] = expf(x[i] - m) * zinv;
+    }
+}
+
 // Streaming loads for data read exactly once.
 __device__ __forceinline__ float4 ld_stream(const float4 *p) { return __ldcs(p); }
 __device__ __forceinline__ float ld_stream(const float *p) { return __ldcs(p); }

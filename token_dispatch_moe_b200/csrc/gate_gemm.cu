@@ -85,20 +85,25 @@ struct RowStats {
     float m, z;  // row max and softmax denominator (when needed)
 };
 
+// Keys of the 16 experts c0 .. c0 + 15 from their logits (the same arithmetic
+// as the route kernels); experts past E get -inf.
 template <bool MONO>
-__device__ __forceinline__ float fused_key(const FusedArgs &f, float l, int e, const RowStats &st,
-                                           float zinv) {
-    if (MONO) return l;
-    float x;
-    if (f.score == MOE_SCORE_SOFTMAX)
-        x = expf(l - st.m) * zinv;
-    else if (f.score == MOE_SCORE_SIGMOID)
-        x = sigmoid_key(l);
-    else if (f.score == MOE_SCORE_SQRT_SOFTPLUS)
-        x = sqrt_softplus_score(l);
-    else
-        x = l;
-    return x + (f.bias ? __ldg(f.bias + e) : 0.0f);
+__device__ __forceinline__ void fused_keys16(const FusedArgs &f, const float (&l)[16], int c0,
+                                             int E, const RowStats &st, float zinv,
+                                             float (&x)[16]) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) x[i] = l[i];
+    if (!MONO) {
+        score_keys<16>(f.score, x, st.m, zinv);
+        if (f.bias) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (c0 + i < E) x[i] += __ldg(f.bias + c0 + i);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        if (c0 + i >= E) x[i] = -INFINITY;
 }
 
 __device__ __forceinline__ uint32_t fkey_bits(float v) {
@@ -137,10 +142,8 @@ __device__ __forceinline__ void chunk_keys(const FusedArgs &f, uint32_t trow, ui
         tmem_ld16_nowait(trow + (uint32_t)c0, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            l[i] = __uint_as_float(r[i]);
-            x[i] = (c0 + i < E) ? fused_key<MONO>(f, l[i], c0 + i, st, zinv) : -INFINITY;
-        }
+        for (int i = 0; i < 16; ++i) l[i] = __uint_as_float(r[i]);
+        fused_keys16<MONO>(f, l, c0, E, st, zinv, x);
     } else {
         tmem_ld16_nowait(trow + koff + (uint32_t)c0, q);
         if (need_logits) tmem_ld16_nowait(trow + (uint32_t)c0, r);
@@ -222,9 +225,12 @@ __device__ __forceinline__ void route_epilogue(const GemmArgs &g, const FusedArg
             uint32_t r[16];
             tmem_ld16_nowait(trow + (uint32_t)c0, r);
             tmem_wait_ld();
+            float l[16], x[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                r[i] = __float_as_uint(fused_key<MONO>(f, __uint_as_float(r[i]), c0 + i, st, zinv));
+            for (int i = 0; i < 16; ++i) l[i] = __uint_as_float(r[i]);
+            fused_keys16<MONO>(f, l, c0, E, st, zinv, x);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(x[i]);
             tmem_st16(trow + koff + (uint32_t)c0, r);
         }
         tmem_wait_st();

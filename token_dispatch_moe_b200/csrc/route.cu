@@ -316,18 +316,6 @@ __device__ __forceinline__ void net_merge(uint32_t (&L)[P], uint32_t &ext, int m
             }
 }
 
-// Selection key of an expert from its logit (the same arithmetic as route_row).
-__device__ __forceinline__ float quad_key(int score, float l, float m, float zinv, float b) {
-    float x = l;
-    if (score == MOE_SCORE_SOFTMAX)
-        x = expf(l - m) * zinv;
-    else if (score == MOE_SCORE_SIGMOID)
-        x = sigmoid_key(l);
-    else if (score == MOE_SCORE_SQRT_SOFTPLUS)
-        x = sqrt_softplus_score(l);
-    return x + b;
-}
-
 // fma(v, 0, acc) turns acc into NaN for a NaN or infinite v.
 __device__ __forceinline__ float finite_acc(float acc, const float4 &v) {
     acc = fmaf(v.x, 0.0f, acc);
@@ -435,10 +423,9 @@ __global__ void __launch_bounds__(kQuadThreads, 3) route_quad_kernel(const __gri
             fin = finite_acc(fin, v);
             if (!mono) {
                 const float4 b = *reinterpret_cast<const float4 *>(bias_s + e0);
-                v.x = quad_key(a.score, v.x, m, zinv, b.x);
-                v.y = quad_key(a.score, v.y, m, zinv, b.y);
-                v.z = quad_key(a.score, v.z, m, zinv, b.z);
-                v.w = quad_key(a.score, v.w, m, zinv, b.w);
+                float x[4] = {v.x, v.y, v.z, v.w};
+                score_keys<4>(a.score, x, m, zinv);  // the same arithmetic as route_row
+                v = make_float4(x[0] + b.x, x[1] + b.y, x[2] + b.z, x[3] + b.w);
                 fin = finite_acc(fin, v);
             }
         };

@@ -243,16 +243,10 @@ __device__ __forceinline__ void route_row(const RouteArgs &a, const float *src, 
     if (a.keys_from_scores) {
         const float zinv = 1.0f / z;
 #pragma unroll
-        for (int s = 0; s < VPL; ++s) {
-            float x = l[s];
-            if (a.score == MOE_SCORE_SOFTMAX)
-                x = expf(l[s] - m) * zinv;
-            else if (a.score == MOE_SCORE_SIGMOID)
-                x = sigmoid_key(l[s]);
-            else if (a.score == MOE_SCORE_SQRT_SOFTPLUS)
-                x = sqrt_softplus_score(l[s]);
-            v[s] = x + biasr[s];
-        }
+        for (int s = 0; s < VPL; ++s) v[s] = l[s];
+        score_keys<VPL>(a.score, v, m, zinv);
+#pragma unroll
+        for (int s = 0; s < VPL; ++s) v[s] += biasr[s];
     } else {
 #pragma unroll
         for (int s = 0; s < VPL; ++s) v[s] = l[s];
