@@ -131,6 +131,49 @@ def test_route_parity(case):
     print(case, r)
 
 
+NEAR_TIE_CASES = [
+    # E, k_max, score, G, TG, topn, logit step giving keys about 2e-5 apart (relative)
+    (128, 4, "topk_softmax", 1, 1, 1, 8e-5),     # keys are the logits
+    (128, 8, "softmax", 1, 1, 1, 8e-5),
+    (256, 8, "sigmoid", 8, 4, 2, 1.1e-3),        # deepseek-v3 layout, scored keys
+    (384, 6, "sqrt_softplus", 4, 2, 2, 1.6e-4),
+]
+
+
+@pytest.mark.parametrize("case", NEAR_TIE_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_route_prefix_near_ties(case):
+    """Rows whose leading experts' keys are 2e-5 apart: closer than the 2^-14
+    relative resolution of the 23-bit key prefix of the selection words, so
+    the rows tie on prefixes and are ordered again on the whole key; wider
+    than the 1e-6 near-tie band, so the order must be exactly the oracle's."""
+    E, k_max, score, G, TG, topn, step = case
+    T = 515
+    g = _gen(E + k_max * 7)
+    logits = torch.randn((T, E), generator=g, device=DEV)
+    rows = torch.arange(0, T, 3, device=DEV)
+    for t in rows.tolist():
+        who = torch.randperm(E, generator=g, device=DEV)[:12]  # ids in random order
+        logits[t, who] = 4.0 + step * torch.arange(12, device=DEV, dtype=torch.float32)
+    p = moe.RouteParams.make(E, k_max, score, G, TG, topn, True, 1.0)
+    ids = torch.full((T, k_max), -7, dtype=torch.int32, device=DEV)
+    w = torch.full((T, k_max), 7.0, device=DEV)
+    st = _status()
+    moe.moe_route(logits, None, None, p, ids, w, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    lg = logits.cpu().numpy()
+    if score in ("topk_softmax", "softmax"):  # keys are the logits: count prefix ties
+        u = lg.view(np.uint32)
+        img = np.where(u >> 31, ~u, u | np.uint32(0x80000000)) >> 9
+        top = np.sort(img, axis=1)[:, ::-1][:, :k_max + 1]
+        tied = (np.diff(top, axis=1) == 0).any(axis=1)
+        assert tied[::3].mean() > 0.5
+    # (a swap is accepted only below a 1e-6 relative key gap: never between
+    # the crafted experts)
+    check_route(ids.cpu().numpy(), w.cpu().numpy(), lg, k_max=k_max, score=score,
+                n_groups=G, topk_groups=TG, group_topn=topn, renormalize=True)
+
+
 def test_route_nan_and_bad_k():
     E, k = 16, 4
     logits = torch.randn((3, E), device=DEV)
