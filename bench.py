@@ -420,6 +420,9 @@ def run_ours(args):
     experts = None
     if args.ffn:
         from token_dispatch_moe_b200.workloads import make_expert_weights
+        if not wl.ffn_dim:
+            raise SystemExit(f"--ffn: {wl.name} has no expert FFN shape; use --workload with one "
+                             f"of {', '.join(n for n, w in WORKLOADS.items() if w.ffn_dim)}")
         wl = wl.with_ffn()
         experts = make_expert_weights(wl, device, seed_offset=rank_seed_offset(rank))
     inp = make_inputs(wl, device, with_y=experts is None, seed_offset=rank_seed_offset(rank))
