@@ -579,6 +579,12 @@ GROUPED_CASES = [
     (100, 8, 1, 2, 2, "softmax", True, 1.0, False),         # one group: the flat rule
     (333, 96, 3, 32, 5, "softmax", True, 1.0, True),        # whole groups: the flat rule
     (200, 30, 3, 2, 4, "softmax", False, 1.0, True),        # E not a multiple of 32
+    # quad path (whole 16-expert chunks and groups, k and k_per_group <= 8)
+    (1003, 256, 16, 1, 8, "sigmoid", True, 2.5, False),     # groups of 16, one candidate each
+    (515, 128, 1, 8, 8, "softmax", True, 1.0, False),       # one group: the flat rule
+    (600, 512, 8, 3, 7, "sqrt_softplus", False, 1.0, False),
+    (300, 128, 8, 2, 4, "topk_softmax", True, 1.0, True),   # integer logits: many ties
+    (70001, 384, 6, 2, 6, "sqrt_softplus", True, 1.0, False),  # more rows than one grid pass
 ]
 
 
