@@ -383,46 +383,44 @@ __global__ void __launch_bounds__(kQuadThreads, 3) route_quad_kernel(const __gri
             __syncwarp();
         }
 
+        auto word = [&](float x, int id) -> uint32_t {
+            if constexpr (FIX)
+                return (__float_as_uint(fmaf(x, fx_scale, fx_off)) << 9) | (uint32_t)(511 - id);
+            else
+                return sel_word(x, id);
+        };
+        // f(keys, first expert) over this lane's vectors of the kept experts
+        auto each_kept = [&](auto &&f) {
+            if (!grouped) {
+#pragma unroll
+                for (int c = 0; c < nch; ++c) {
+                    const int e0 = 16 * c + 4 * j;
+                    if (e0 < E) f(buf[c * 32], e0);
+                }
+            } else {
+                uint32_t mk = kept;
+                for (int gi = 0; gi < a.TG; ++gi) {
+                    const int g = __ffs(mk) - 1;
+                    mk &= mk - 1u;
+                    for (int cc = 0; cc < cpg; ++cc) {
+                        const int c = g * cpg + cc;
+                        const int e0 = 16 * c + 4 * j;
+                        if (e0 < E) f(buf[c * 32], e0);
+                    }
+                }
+            }
+        };
         // select: the P largest words of the kept experts, and the largest
         // word beyond them
         uint32_t L[P];
         uint32_t ext = 0u;
 #pragma unroll
         for (int p = 0; p < P; ++p) L[p] = 0u;
-        auto insert4 = [&](const float4 &v, int e0) {
-            if constexpr (FIX) {
-                auto fw = [&](float x, int id) {
-                    return (__float_as_uint(fmaf(x, fx_scale, fx_off)) << 9) | (uint32_t)(511 - id);
-                };
-                net_insert4<P>(L, ext, fw(v.x, e0), fw(v.y, e0 + 1), fw(v.z, e0 + 2),
-                               fw(v.w, e0 + 3));
-            } else {
-                net_insert4<P>(L, ext, sel_word(v.x, e0), sel_word(v.y, e0 + 1),
-                               sel_word(v.z, e0 + 2), sel_word(v.w, e0 + 3));
-            }
-        };
-        if (!grouped) {
-#pragma unroll
-            for (int c = 0; c < nch; ++c) {
-                const int e0 = 16 * c + 4 * j;
-                if (e0 < E) {
-                    const float4 v = buf[c * 32];
-                    if (mono) fin = finite_acc(fin, v);  // (keys were checked above)
-                    insert4(v, e0);
-                }
-            }
-        } else {
-            uint32_t mk = kept;
-            for (int gi = 0; gi < a.TG; ++gi) {
-                const int g = __ffs(mk) - 1;
-                mk &= mk - 1u;
-                for (int cc = 0; cc < cpg; ++cc) {
-                    const int c = g * cpg + cc;
-                    const int e0 = 16 * c + 4 * j;
-                    if (e0 < E) insert4(buf[c * 32], e0);
-                }
-            }
-        }
+        each_kept([&](const float4 &v, int e0) {
+            if (mono && !grouped) fin = finite_acc(fin, v);  // (other keys were checked above)
+            net_insert4<P>(L, ext, word(v.x, e0), word(v.y, e0 + 1), word(v.z, e0 + 2),
+                           word(v.w, e0 + 3));
+        });
         net_merge<P>(L, ext, 1);
         net_merge<P>(L, ext, 2);
         // check: distinct selected prefixes, and the next word's prefix below
