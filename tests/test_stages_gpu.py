@@ -417,7 +417,9 @@ def test_dispatch_limited_then_permute_combine():
 
 @pytest.mark.parametrize("T,k,d,E", [(1, 1, 8, 4), (999, 8, 2048, 64), (500, 6, 7168, 384),
                                      (1234, 4, 2880, 128), (100, 32, 136, 512),
-                                     (257, 2, 128, 8)])
+                                     (257, 2, 128, 8),
+                                     # several rows a warp through both row buffers
+                                     (10007, 3, 2048, 64), (2000, 8, 7168, 256)])
 def test_permute_combine_parity(T, k, d, E):
     g = _gen(T * 3 + d)
     ids = torch.randint(0, E, (T, k), generator=g, device=DEV, dtype=torch.int32)
