@@ -196,7 +196,8 @@ moe_status moe_hash_route(const int32_t *token_ids, const int32_t *tid2eid, int3
 
 /*
  * moe_dispatch_workspace_size -- bytes of device scratch moe_dispatch needs for
- * T tokens, k_max slots and E experts (depends only on T*k_max and E).
+ * T tokens, k_max slots and E experts (depends only on T*k_max and E; never
+ * more than 606,208 bytes: at most 296 segments of E rounded up to 4 int32).
  */
 moe_status moe_dispatch_workspace_size(int64_t T, int32_t k_max, int32_t E, size_t *bytes);
 
@@ -264,11 +265,12 @@ moe_status moe_dispatch_limited(const int32_t *topk_ids, int64_t T, int32_t k_ma
  * that owns every device allocation, or code that must avoid the implicit
  * device synchronisation of cudaMalloc.)
  * Same arguments, outputs and status rules as moe_dispatch, minus workspace and
- * ws_bytes.  Its scratch is a 4 MiB array inside the library, held by every GPU
- * that loads the library until the process exits; sizes whose
- * moe_dispatch_workspace_size() exceeds 4 MiB are rejected with
- * MOE_ERR_UNSUPPORTED and nothing is launched.  The library allocates and frees
- * nothing here either.
+ * ws_bytes.  Its scratch is a 606,208-byte array inside the library (the most
+ * moe_dispatch_workspace_size() returns for any size it accepts: 296 segments
+ * x 512 experts x 4 bytes), held by every GPU that loads the library until the
+ * process exits; so every size moe_dispatch accepts fits, and the sizes it
+ * refuses (T*k_max >= 2^31) are refused here the same way, with nothing
+ * launched.  The library allocates and frees nothing here either.
  * The scratch array's device address is looked up (cudaGetSymbolAddress) by
  * the first call in each CUDA context and cached under that context's unique
  * id, so a context destroyed and created again (e.g. after cudaDeviceReset) is

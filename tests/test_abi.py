@@ -50,12 +50,17 @@ def test_status_strings(lib):
 def _expected_workspace(T, k, E):
     """One int32 per (segment, expert), the expert row padded to whole 16-byte
     quads; a segment is 8 warps x 32 lanes x `items` slots, items the smallest
-    of 4, 8, 16 for which 148 segments cover every slot; rounded up to 256 B."""
+    of 4, 8, 16 for which 148 segments cover every slot; above 296 segments a
+    segment takes as many such rounds as keep the segments at most 296;
+    rounded up to 256 B."""
     n = T * k
     items = 4
     while items * 32 * 8 * 148 < n and items < 16:
         items *= 2
-    segs = -(-n // (items * 32 * 8))
+    seg = items * 32 * 8
+    s1 = -(-n // seg)
+    rounds = 1 if s1 <= 296 else -(-s1 // 296)
+    segs = -(-n // (seg * rounds))
     b = segs * (-(-E // 4) * 4) * 4
     return -(-b // 256) * 256
 
@@ -67,6 +72,11 @@ def test_workspace_size(lib):
         assert moe.moe_dispatch_workspace_size(T, k, E) == _expected_workspace(T, k, E)
     assert moe.moe_dispatch_workspace_size(16384, 16, 128) == 128 * 128 * 4  # 128 segments of 8 items
     assert moe.moe_dispatch_workspace_size(1, 1, 1) == 256
+    # rounds keep the segments at most 296, whatever the size
+    assert moe.moe_dispatch_workspace_size(37888, 32, 512) == 296 * 512 * 4  # exactly 296
+    assert moe.moe_dispatch_workspace_size(65536, 32, 512) == 256 * 512 * 4  # 512 -> 2 rounds
+    for T in (37889, 262144, 1 << 22, (2 ** 31 - 1) // 32):
+        assert moe.moe_dispatch_workspace_size(T, 32, 512) <= 296 * 512 * 4
     with pytest.raises(moe.MoeError):
         moe.moe_dispatch_workspace_size(10, 33, 8)   # k_max > 32
     with pytest.raises(moe.MoeError):
@@ -99,6 +109,14 @@ def test_host_validation_needs_no_gpu(lib):
         moe.MOE_ERR_INVALID_ARG
     assert lib.moe_dispatch(bad, 4, 2, 8, bad, bad, bad, bad, ctypes.c_void_p(256), 0, None,
                             None) == moe.MOE_ERR_INVALID_ARG  # workspace too small
+
+
+def test_static_dispatch_refuses_without_launch(lib):
+    """The only sizes moe_dispatch_static refuses are those moe_dispatch refuses
+    (T*k_max >= 2^31): answered before any device call (pointers never read)."""
+    bad = ctypes.c_void_p(16)
+    assert lib.moe_dispatch_static(bad, 1 << 26, 32, 512, bad, bad, bad, bad, None,
+                                   None) == moe.MOE_ERR_UNSUPPORTED
 
 
 def test_binding_fails_loudly_without_library(tmp_path):

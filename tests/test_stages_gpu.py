@@ -312,7 +312,9 @@ def _dispatch(ids, E):
     (25000, 8, 128, 0.3, True), (4000, 5, 130, 0.1, False),
     # around the one-block launch (at most 1024 slots)
     (128, 8, 64, 0.1, True), (1024, 1, 64, 0.1, True), (1025, 1, 16, 0.0, True),
-    (512, 8, 64, 0.1, True)])
+    (512, 8, 64, 0.1, True),
+    # over 296 segments of 4096 slots: segments of 2 and 7 rounds, ragged last round
+    (200003, 8, 256, 0.1, True), (40001, 32, 512, 0.05, False), (1048577, 8, 128, 0.0, True)])
 def test_dispatch_parity(T, k, E, empty_frac, hot):
     g = _gen(T + k + E)
     ids = torch.randint(0, E, (T, k), generator=g, device=DEV, dtype=torch.int32)
@@ -350,7 +352,9 @@ def test_dispatch_edge_cases():
     (1, 1, 4, 0, 1, False), (3001, 1, 128, 0, 128, True), (70000, 1, 128, 547, 128, True),
     (5000, 8, 64, 400, 16, False), (777, 6, 384, 3, 1, True), (40000, 4, 128, 1, 7, True),
     (20000, 16, 512, 0, 64, False), (9000, 2, 8, 2250, 128, True),
-    (200, 2, 8, 0, 4096, False), (3000, 32, 16, 5, 1, True)])
+    (200, 2, 8, 0, 4096, False), (3000, 32, 16, 5, 1, True),
+    # segments of several rounds, with capacity and padding
+    (200003, 8, 256, 5000, 128, True), (160001, 8, 64, 0, 1, False)])
 def test_dispatch_limited_parity(T, k, E, cap, pad, hot):
     """Capacity cut and block padding, bit-exact against the oracle."""
     g = _gen(T * 7 + E + cap + pad)

@@ -24,6 +24,11 @@
 //               its ids in order, ranking each slot among its peers with the
 //               same id (popcount of lower lanes in the match mask), writing
 //               sorted_token and dest_pos.
+// Above 296 segments of 16 items a lane (1,212,416 slots) each segment takes
+// several rounds of 4096 slots (its block carries per-expert running counts
+// from round to round), so S stays at most 296 and the totals each scatter
+// block sums stay bounded (without rounds, 8 M slots measured 2.4x the time
+// of 4 M, from re-summing S x E totals).
 // Workspace: seg_total [S][Ep] int32, Ep = E rounded up to a multiple of 4.
 #include <cuda.h>
 
@@ -45,8 +50,19 @@ int warp_items(int64_t n_flat) {
     return items;
 }
 
-int64_t num_segments(int64_t n_flat, int items) {
+// Above kMaxSegments segments of 16 items a lane (1,212,416 slots) a segment
+// takes several rounds of 8 warps x 16 items x 32 lanes, so that the totals
+// every scatter block sums (segments x experts) stay bounded.
+constexpr int64_t kMaxSegments = 2 * 148;
+
+int seg_rounds(int64_t n_flat, int items) {
     const int64_t seg = (int64_t)items * 32 * kDispWarps;
+    const int64_t s1 = (n_flat + seg - 1) / seg;
+    return s1 <= kMaxSegments ? 1 : (int)((s1 + kMaxSegments - 1) / kMaxSegments);
+}
+
+int64_t num_segments(int64_t n_flat, int items) {
+    const int64_t seg = (int64_t)items * 32 * kDispWarps * seg_rounds(n_flat, items);
     return (n_flat + seg - 1) / seg;
 }
 
@@ -63,26 +79,35 @@ __device__ __forceinline__ int load_id(const int32_t *ids, int64_t a, int64_t n_
     return e;
 }
 
+// The first slot of warp `warp`'s sub-segment in round r of segment s.
+template <int ITEMS>
+__device__ __forceinline__ int64_t round_base(int64_t s, int rounds, int r, int warp) {
+    return ((s * rounds + r) * kDispWarps + warp) * (int64_t)ITEMS * 32;
+}
+
 template <int ITEMS>
 __global__ void __launch_bounds__(kDispWarps * 32)
     dispatch_count_kernel(const int32_t *__restrict__ ids, int64_t n_flat, int E, int Ep,
-                          int32_t *__restrict__ seg_total, int32_t *status) {
+                          int rounds, int32_t *__restrict__ seg_total, int32_t *status) {
     __shared__ int32_t hist[kMaxE];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t s = blockIdx.x;
     for (int e = threadIdx.x; e < Ep; e += blockDim.x) hist[e] = 0;
     __syncthreads();
     griddep_wait();
-    const int64_t base = (s * kDispWarps + warp) * (int64_t)ITEMS * 32;
     bool bad = false;
-    int eb[ITEMS];  // every load of the sub-segment is issued before any is used
+    for (int r = 0; r < rounds; ++r) {
+        const int64_t base = round_base<ITEMS>(s, rounds, r, warp);
+        int eb[ITEMS];  // every load of the sub-segment is issued before any is used
 #pragma unroll
-    for (int j = 0; j < ITEMS; ++j) eb[j] = load_id(ids, base + (int64_t)j * 32 + lane, n_flat, E, bad);
+        for (int j = 0; j < ITEMS; ++j)
+            eb[j] = load_id(ids, base + (int64_t)j * 32 + lane, n_flat, E, bad);
 #pragma unroll
-    for (int j = 0; j < ITEMS; ++j) {
-        const int e = eb[j];
-        const unsigned peers = __match_any_sync(MOE_FULL_MASK, e);
-        if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[e], __popc(peers));
+        for (int j = 0; j < ITEMS; ++j) {
+            const int e = eb[j];
+            const unsigned peers = __match_any_sync(MOE_FULL_MASK, e);
+            if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[e], __popc(peers));
+        }
     }
     if (__any_sync(MOE_FULL_MASK, bad) && lane == 0) report(status, MOE_ERR_DEVICE_INDEX);
     __syncthreads();
@@ -105,22 +130,21 @@ struct ScatterSmem {
     int32_t hist[kDispWarps][kMaxE];   // per-warp histograms, then each warp's first rank
     int32_t wsum[kDispWarps];
     int32_t kept[kMaxE];               // with limits: kept slots per expert
+    int32_t racc[kMaxE];               // slots of each expert in this segment's earlier rounds
     int32_t drop;
 };
 
-// The scatter of segment s (of S) once sh.total, sh.before and the warps'
-// histograms are in place: exclusive scan of the expert blocks into offsets
-// (segment 0 writes counts, offsets and the dropped count), the padding rows
-// of padded blocks, each warp's first rank per expert, and the stable scatter
-// of the warp's slots (ids eb, peer masks pm, in registers).
-template <int ITEMS, bool LIMITED>
-__device__ __forceinline__ void scatter_tail(ScatterSmem &sh, int64_t s, int64_t S,
-                                             int64_t base, int64_t n_flat, int k_max, int E,
-                                             const int (&eb)[ITEMS], const unsigned (&pm)[ITEMS],
-                                             int32_t *__restrict__ counts,
-                                             int32_t *__restrict__ offsets,
-                                             int32_t *__restrict__ sorted_token,
-                                             int32_t *__restrict__ dest_pos, const Limits &lim) {
+// Segment s (of S) once sh.total holds the per-expert totals: exclusive scan
+// of the expert blocks (the totals, or with limits the kept slots rounded up
+// to the padding) into offsets, left in sh.total; segment 0 writes counts,
+// offsets and the dropped count; with padding, the padding rows of the expert
+// blocks (experts shared out over the segments).
+template <bool LIMITED>
+__device__ __forceinline__ void scatter_offsets(ScatterSmem &sh, int64_t s, int64_t S, int E,
+                                                int32_t *__restrict__ counts,
+                                                int32_t *__restrict__ offsets,
+                                                int32_t *__restrict__ sorted_token,
+                                                const Limits &lim) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     // Exclusive scan of the block sizes (the totals, or with limits the kept
     // slots rounded up to the padding) into offsets: thread i owns experts 2i,
@@ -183,17 +207,31 @@ __device__ __forceinline__ void scatter_tail(ScatterSmem &sh, int64_t s, int64_t
                 sorted_token[p] = -1;
         }
     }
-    // Each warp's first rank per expert, in place of its histogram: earlier
-    // segments + earlier warps of this segment; without limits the block
-    // offset is folded in as well.
+}
+
+// One round of a segment once the warps' histograms of the round are in
+// place: each warp's first rank per expert (earlier segments, earlier rounds
+// of this segment, earlier warps of this round; without limits the block
+// offset as well), then the stable scatter of the warp's slots (ids eb, peer
+// masks pm, in registers).  Leaves sh.racc counting this round too.
+template <int ITEMS, bool LIMITED>
+__device__ __forceinline__ void scatter_round(ScatterSmem &sh, int64_t base, int64_t n_flat,
+                                              int k_max, int E, const int (&eb)[ITEMS],
+                                              const unsigned (&pm)[ITEMS],
+                                              int32_t *__restrict__ sorted_token,
+                                              int32_t *__restrict__ dest_pos, const Limits &lim) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int32_t b = (LIMITED ? 0 : sh.total[e]) + sh.before[e];
+        int32_t b = (LIMITED ? 0 : sh.total[e]) + sh.before[e] + sh.racc[e];
+        int32_t here = 0;
 #pragma unroll
         for (int w = 0; w < kDispWarps; ++w) {
             const int32_t h = sh.hist[w][e];
             sh.hist[w][e] = b;
             b += h;
+            here += h;
         }
+        sh.racc[e] += here;
     }
     __syncthreads();
 
@@ -221,7 +259,7 @@ __device__ __forceinline__ void scatter_tail(ScatterSmem &sh, int64_t s, int64_t
 template <int ITEMS, bool LIMITED>
 __global__ void __launch_bounds__(kDispWarps * 32)
     dispatch_scatter_kernel(const int32_t *__restrict__ ids, int64_t n_flat, int k_max, int E,
-                            int Ep, int64_t S, const int32_t *__restrict__ seg_total,
+                            int Ep, int64_t S, int rounds, const int32_t *__restrict__ seg_total,
                             int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
                             int32_t *__restrict__ sorted_token, int32_t *__restrict__ dest_pos,
                             Limits lim) {
@@ -232,14 +270,16 @@ __global__ void __launch_bounds__(kDispWarps * 32)
     for (int e = threadIdx.x; e < Ep; e += blockDim.x) {
         sh.total[e] = 0;
         sh.before[e] = 0;
+        sh.racc[e] = 0;
     }
     for (int i = threadIdx.x; i < kDispWarps * Ep; i += blockDim.x) sh.hist[i / Ep][i % Ep] = 0;
     __syncthreads();
     griddep_wait();
 
-    // This warp's ids: loaded once, kept in registers for both passes below.
-    // An id outside [-1, E) counts as empty here; the count kernel reported it.
-    const int64_t base = (s * kDispWarps + warp) * (int64_t)ITEMS * 32;
+    // This warp's ids of the first round, loaded while the totals below are
+    // summed.  An id outside [-1, E) counts as empty here; the count kernel
+    // reported it.
+    int64_t base = round_base<ITEMS>(s, rounds, 0, warp);
     bool bad = false;
     int eb[ITEMS];
 #pragma unroll
@@ -287,19 +327,35 @@ __global__ void __launch_bounds__(kDispWarps * 32)
         }
     }
 
-    // This warp's histogram, from the ids in registers (one leader per id).
-    unsigned pm[ITEMS];
-#pragma unroll
-    for (int j = 0; j < ITEMS; ++j) {
-        const int e = eb[j];
-        pm[j] = __match_any_sync(MOE_FULL_MASK, e);
-        if (e >= 0 && lane == __ffs(pm[j]) - 1) sh.hist[warp][e] += __popc(pm[j]);
-        __syncwarp();
-    }
     __syncthreads();
+    scatter_offsets<LIMITED>(sh, s, S, E, counts, offsets, sorted_token, lim);
 
-    scatter_tail<ITEMS, LIMITED>(sh, s, S, base, n_flat, k_max, E, eb, pm, counts, offsets,
-                                 sorted_token, dest_pos, lim);
+    for (int r = 0; r < rounds; ++r) {
+        if (r > 0) {
+            base = round_base<ITEMS>(s, rounds, r, warp);
+#pragma unroll
+            for (int j = 0; j < ITEMS; ++j)
+                eb[j] = load_id(ids, base + (int64_t)j * 32 + lane, n_flat, E, bad);
+            // the last round's running ranks are done with: fresh histograms
+            for (int i = threadIdx.x; i < kDispWarps * Ep; i += blockDim.x)
+                sh.hist[i / Ep][i % Ep] = 0;
+            __syncthreads();
+        }
+        // This warp's histogram of the round, from the ids in registers (one
+        // leader per id).
+        unsigned pm[ITEMS];
+#pragma unroll
+        for (int j = 0; j < ITEMS; ++j) {
+            const int e = eb[j];
+            pm[j] = __match_any_sync(MOE_FULL_MASK, e);
+            if (e >= 0 && lane == __ffs(pm[j]) - 1) sh.hist[warp][e] += __popc(pm[j]);
+            __syncwarp();
+        }
+        __syncthreads();
+        scatter_round<ITEMS, LIMITED>(sh, base, n_flat, k_max, E, eb, pm, sorted_token, dest_pos,
+                                      lim);
+        __syncthreads();
+    }
     griddep_launch_dependents();
 }
 
@@ -340,10 +396,11 @@ __global__ void __launch_bounds__(kDispWarps * 32)
         for (int w = 0; w < kDispWarps; ++w) c += sh.hist[w][e];
         sh.total[e] = c;
         sh.before[e] = 0;
+        sh.racc[e] = 0;
     }
     __syncthreads();
-    scatter_tail<ITEMS, LIMITED>(sh, 0, 1, base, n_flat, k_max, E, eb, pm, counts, offsets,
-                                 sorted_token, dest_pos, lim);
+    scatter_offsets<LIMITED>(sh, 0, 1, E, counts, offsets, sorted_token, lim);
+    scatter_round<ITEMS, LIMITED>(sh, base, n_flat, k_max, E, eb, pm, sorted_token, dest_pos, lim);
     griddep_launch_dependents();
 }
 
@@ -353,7 +410,7 @@ __global__ void __launch_bounds__(kDispWarps * 32)
 // blocks and two launches), else count + scatter over S segments of `items`
 // items a lane (segment totals in the workspace).
 template <bool LIMITED>
-cudaError_t launch_dispatch(int items, int64_t S, cudaStream_t cs, const int32_t *ids,
+cudaError_t launch_dispatch(int items, int rounds, int64_t S, cudaStream_t cs, const int32_t *ids,
                             int64_t n_flat, int k_max, int E, int32_t *seg_total,
                             int32_t *counts, int32_t *offsets, int32_t *sorted_token,
                             int32_t *dest_pos, int32_t *d_status, Limits lim) {
@@ -367,10 +424,10 @@ cudaError_t launch_dispatch(int items, int64_t S, cudaStream_t cs, const int32_t
 #define MOE_DISPATCH_CASE(IT)                                                                     \
     case IT:                                                                                      \
         err = launch_pdl(dispatch_count_kernel<IT>, grid, block, 0, cs, ids, n_flat, E, Ep,       \
-                         seg_total, d_status);                                                    \
+                         rounds, seg_total, d_status);                                            \
         if (err != cudaSuccess) return err;                                                       \
         return launch_pdl(dispatch_scatter_kernel<IT, LIMITED>, grid, block, 0, cs, ids, n_flat,  \
-                          k_max, E, Ep, S, (const int32_t *)seg_total, counts, offsets,           \
+                          k_max, E, Ep, S, rounds, (const int32_t *)seg_total, counts, offsets,   \
                           sorted_token, dest_pos, lim);
     switch (items) {
         MOE_DISPATCH_CASE(4)
@@ -416,7 +473,7 @@ extern "C" moe_status moe_dispatch(const int32_t *topk_ids, int64_t T, int32_t k
     const int items = warp_items(n_flat);
     const int64_t S = num_segments(n_flat, items);
     if (S > 0) {
-        if (launch_dispatch<false>(items, S, cs, topk_ids, n_flat, (int)k_max, (int)E,
+        if (launch_dispatch<false>(items, seg_rounds(n_flat, items), S, cs, topk_ids, n_flat, (int)k_max, (int)E,
                                    static_cast<int32_t *>(workspace), counts, offsets,
                                    sorted_token, dest_pos, d_status,
                                    Limits{INT32_MAX, 1, nullptr}) != cudaSuccess) {
@@ -476,7 +533,7 @@ extern "C" moe_status moe_dispatch_limited(const int32_t *topk_ids, int64_t T, i
     const int64_t S = num_segments(n_flat, items);
     if (S > 0) {
         const Limits lim{capacity > 0 ? capacity : INT32_MAX, pad, dropped};
-        if (launch_dispatch<true>(items, S, cs, topk_ids, n_flat, (int)k_max, (int)E,
+        if (launch_dispatch<true>(items, seg_rounds(n_flat, items), S, cs, topk_ids, n_flat, (int)k_max, (int)E,
                                   static_cast<int32_t *>(workspace), counts, offsets, sorted_token,
                                   dest_pos, d_status, lim) != cudaSuccess) {
             cudaGetLastError();
@@ -505,7 +562,11 @@ extern "C" moe_status moe_dispatch_limited(const int32_t *topk_ids, int64_t T, i
 // an address of the old one.
 namespace moe {
 namespace {
-constexpr size_t kStaticScratchBytes = size_t(4) << 20;
+// The most moe_dispatch_workspace_size() returns for any size it accepts:
+// kMaxSegments segments of 512 experts (606,208 bytes), so no accepted size is
+// refused for want of scratch.
+constexpr size_t kStaticScratchBytes = size_t(kMaxSegments) * kMaxE * sizeof(int32_t);
+static_assert(kStaticScratchBytes % 256 == 0, "workspace sizes are rounded to 256 bytes");
 constexpr int kScratchCacheSlots = 64;
 
 typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
@@ -589,7 +650,7 @@ extern "C" moe_status moe_dispatch_static(const int32_t *topk_ids, int64_t T, in
     size_t need = 0;
     moe_status st = moe_dispatch_workspace_size(T, k_max, E, &need);
     if (st != MOE_OK) return st;
-    if (need > kStaticScratchBytes) return MOE_ERR_UNSUPPORTED;  // beyond the fixed scratch
+    if (need > kStaticScratchBytes) return MOE_ERR_UNSUPPORTED;  // (cannot happen: see above)
     void *addr = static_scratch();
     if (!addr) return MOE_ERR_CUDA;
     // Every scratch entry a dispatch reads is written earlier by the same
