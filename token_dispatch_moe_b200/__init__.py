@@ -417,8 +417,9 @@ def moe_wait_probe(limit_ns: int, d_status, d_outcome=None, stream=None):
 
 def moe_dispatch_static(topk_ids, E, counts, offsets, sorted_token, dest_pos, d_status=None,
                         stream=None):
-    """moe_dispatch with the library's own fixed 4 MiB scratch instead of a
-    caller-allocated workspace, for callers that cannot allocate device memory.
+    """moe_dispatch with the library's own fixed scratch (606,208 bytes: the
+    largest workspace any accepted size needs) instead of a caller-allocated
+    workspace, for callers that cannot allocate device memory.
     Calls that overlap on the GPU race on that scratch; the first call on a
     device should come before any stream capture."""
     _need(topk_ids, torch.int32, "topk_ids", 2)
