@@ -161,12 +161,14 @@ moe_status run_permute(const moe_bf16_t *x, const int32_t *dest_pos, int64_t T, 
     if (T == 0 || k_max == 0) return MOE_OK;
     if (!x || !dest_pos || !xs || !aligned16(x) || !aligned16(xs)) return MOE_ERR_INVALID_ARG;
     if (T * (int64_t)k_max >= (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
-    // Sixteen vectors per lane on wide rows (d >= 4096): more bytes in flight
-    // per warp measured 0.6-1.1 % faster there; eight elsewhere.
+    // Sixteen vectors per lane on rows of more than 256 vectors (d > 2048): more
+    // bytes in flight per warp measured 0.6-1.1 % faster at d >= 4096, and at
+    // d = 2880 (360 vectors) one round of sixteen instead of a full round of
+    // eight and a third of one measured 1289 -> 1225 us; eight elsewhere.
     const uint4 *x4 = reinterpret_cast<const uint4 *>(x);
     uint4 *xs4 = reinterpret_cast<uint4 *>(xs);
     const cudaError_t err =
-        d / 8 >= 512 ? launch_rows(permute_kernel<16, CHECK>, row_grid(T), as_cuda(stream), x4,
+        d / 8 > 256 ? launch_rows(permute_kernel<16, CHECK>, row_grid(T), as_cuda(stream), x4,
                                    dest_pos, T, (int)k_max, d / 8, xs4, rows, d_status)
                      : launch_rows(permute_kernel<8, CHECK>, row_grid(T), as_cuda(stream), x4,
                                    dest_pos, T, (int)k_max, d / 8, xs4, rows, d_status);
