@@ -184,10 +184,17 @@ moe_status run_permute(const moe_bf16_t *x, const int32_t *dest_pos, int64_t T, 
     // bytes in flight per warp measured 0.6-1.1 % faster at d >= 4096, and at
     // d = 2880 (360 vectors) one round of sixteen instead of a full round of
     // eight and a third of one measured 1289 -> 1225 us; eight elsewhere.
+    // Rows of 769-896 vectors (d = 7168: deepseek-v3/v4) take twenty-eight, the
+    // whole row in one round (133 registers, one block an SM): 1343 -> 1312 us
+    // and 1048 -> 1026 us; capped at 128 registers for two blocks an SM it
+    // spilled and measured 1331 us; twenty at d = 5120 gained nothing.
     const uint4 *x4 = reinterpret_cast<const uint4 *>(x);
     uint4 *xs4 = reinterpret_cast<uint4 *>(xs);
     const cudaError_t err =
-        d / 8 > 256 ? launch_rows(permute_kernel<16, CHECK>, row_grid(T), as_cuda(stream), x4,
+        (d / 8 > 768 && d / 8 <= 896)
+            ? launch_rows(permute_kernel<28, CHECK>, row_grid(T), as_cuda(stream), x4, dest_pos, T,
+                          (int)k_max, d / 8, xs4, rows, d_status)
+        : d / 8 > 256 ? launch_rows(permute_kernel<16, CHECK>, row_grid(T), as_cuda(stream), x4,
                                    dest_pos, T, (int)k_max, d / 8, xs4, rows, d_status)
                      : launch_rows(permute_kernel<8, CHECK>, row_grid(T), as_cuda(stream), x4,
                                    dest_pos, T, (int)k_max, d / 8, xs4, rows, d_status);
