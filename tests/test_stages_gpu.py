@@ -174,6 +174,29 @@ def test_route_prefix_near_ties(case):
                 n_groups=G, topk_groups=TG, group_topn=topn, renormalize=True)
 
 
+@pytest.mark.parametrize("spread", [50.0, 1e-3])
+def test_route_fixed_point_words_bias_range(spread):
+    """Sigmoid keys with a bias spread far wider (50) and far narrower (1e-3)
+    than the scores: the fixed-point selection words scale to the bias range,
+    so their step is coarse in the first case (many prefix ties, settled by the
+    exact routine) and fine in the second."""
+    T, E, k = 1003, 256, 8
+    g = _gen(int(spread * 1000) + 7)
+    logits = torch.randn((T, E), generator=g, device=DEV) * 2
+    bias = (torch.rand((E,), generator=g, device=DEV) * 2 - 1) * spread
+    bias[::37] = bias[0]  # some equal biases
+    p = moe.RouteParams.make(E, k, "sigmoid", 8, 4, 2, True, 2.5)
+    ids = torch.full((T, k), -7, dtype=torch.int32, device=DEV)
+    w = torch.full((T, k), 7.0, device=DEV)
+    st = _status()
+    moe.moe_route(logits, bias, None, p, ids, w, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    check_route(ids.cpu().numpy(), w.cpu().numpy(), logits.cpu().numpy(), k_max=k,
+                score="sigmoid", bias=bias.cpu().numpy(), n_groups=8, topk_groups=4,
+                group_topn=2, renormalize=True, route_scale=2.5)
+
+
 def test_route_nan_and_bad_k():
     E, k = 16, 4
     logits = torch.randn((3, E), device=DEV)
