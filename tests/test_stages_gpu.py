@@ -656,6 +656,44 @@ def test_route_grouped_parity(case):
         assert torch.equal(fids, ids)
 
 
+@pytest.mark.parametrize("E,G,kpg,k", [(128, 8, 2, 4),    # quad kernel
+                                      (30, 3, 2, 4)])    # warp kernel
+def test_route_grouped_nan_logits(E, G, kpg, k):
+    """A NaN logit ranks below every number, as the header states (the
+    ranking is of the logits, which every score orders alike), and the call
+    reports MOE_ERR_NAN_LOGIT.  The ids of NaN rows are checked against that
+    rule written out here; rows without NaN against the oracle."""
+    T = 64
+    g = _gen(E + G)
+    logits = torch.randn((T, E), generator=g, device=DEV)
+    nan_rows = [1, 7, 30]
+    logits[1, 5] = float("nan")
+    logits[7, :E // G] = float("nan")  # a whole group
+    logits[30, ::3] = float("nan")
+    p = moe.RouteParams.make(E, k, "softmax", G, 1, 1, True, 1.0)
+    ids = torch.full((T, k), -7, dtype=torch.int32, device=DEV)
+    w = torch.full((T, k), 7.0, device=DEV)
+    st = _status()
+    moe.moe_route_grouped(logits, p, kpg, ids, w, st)
+    torch.cuda.synchronize()
+    assert st.item() == moe.MOE_ERR_NAN_LOGIT
+    lg, gi = logits.cpu().numpy(), ids.cpu().numpy()
+    gsz = E // G
+    order = lambda e, row: (0 if np.isnan(row[e]) else 1, -np.inf if np.isnan(row[e]) else row[e], -e)  # noqa: E731
+    for t in nan_rows:
+        row = lg[t]
+        cand = []
+        for q in range(G):
+            grp = sorted(range(q * gsz, (q + 1) * gsz), key=lambda e: order(e, row), reverse=True)
+            cand += grp[:kpg]
+        want = sorted(cand, key=lambda e: order(e, row), reverse=True)[:k]
+        assert gi[t].tolist() == want, (t, gi[t], want)
+    ok = np.array([t not in nan_rows for t in range(T)])
+    o = oracle.route_grouped(lg[ok], k_max=k, score=oracle.SOFTMAX, n_groups=G, k_per_group=kpg,
+                             renormalize=True, route_scale=1.0, want_keys=True)
+    assert np.array_equal(gi[ok], o["ids"])
+
+
 def test_route_grouped_validation():
     logits = torch.zeros((4, 16), device=DEV)
     ids = torch.empty((4, 4), dtype=torch.int32, device=DEV)
