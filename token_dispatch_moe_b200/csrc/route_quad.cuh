@@ -383,6 +383,8 @@ __global__ void __launch_bounds__(kQuadThreads, 3) route_quad_kernel(const __gri
             __syncwarp();
         }
 
+        // the selection word of key x of expert id: a fixed-point (FIX) or
+        // float-image prefix above 511 - id
         auto word = [&](float x, int id) -> uint32_t {
             if constexpr (FIX)
                 return (__float_as_uint(fmaf(x, fx_scale, fx_off)) << 9) | (uint32_t)(511 - id);
